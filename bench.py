@@ -1,0 +1,476 @@
+#!/usr/bin/env python
+"""Decode throughput of the group-wise 4-bit OPT-style block on B200.
+
+Default workload: the OPT-30B shape (48 layers, h=7168, 56 heads, FFN 28672,
+vocab 50272), weights and KV cache in the group-wise 4-bit format, a block of
+144 sequences, prompt length 512, 32 generated tokens, one GPU batch of 144.
+
+One timed step is the decode phase of flexq_generate: the n-1 = 31 decode
+columns of the zig-zag block (every layer for every GPU batch, then the tied
+LM head and the greedy choice), run through the public entry point
+flexq_generate_decode on caches filled by one prefill.  value = b * (n - 1) *
+n_gpus / (max over ranks of the step time).  Weights (16.7 GB) and KV (30 GB)
+are far larger than L2, so no flush is needed between steps.
+
+Other figures on the same JSON line: the prefill column timed once, the
+per-kernel breakdown of one profiled decode step (CUDA events around every
+kernel, a separate pass after the timed steps), the roofline of the dominant
+kernel against MEASURED_PEAKS.json, SM clocks sampled during the timed
+region, an end-to-end run of flexq_generate with the prompts uploaded from
+pinned host memory and the tokens read back, and the CPU oracle timed on a
+bounded sample (`cpu_baseline`).
+
+`--impl reference` times the CPU oracle alone on the same metric (each step =
+one oracle layer decode for a few sequences, extrapolated to tokens/s).
+Multi-GPU: one independent replica per rank (weak scaling, no collective on
+the data path; torch.distributed only for the barrier and the max-over-ranks
+timing).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+
+# ---------------------------------------------------------------------------
+# common helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "quantized_opt_decode_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kind: str):
+    """DRAM bytes per launch of `kind` from the committed ncu summary, or None
+    when absent or taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = csrc_hash()
+    with open(path) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 3 and not line.startswith("#") and parts[0] == kind:
+                return float(parts[1]) if parts[2] == cur else None
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while active."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = num(rows[0][2])
+        load = [v for v in sm if smax and v > 0.5 * smax] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per kernel call (decode step, M = b rows)
+# ---------------------------------------------------------------------------
+def kernel_work(p: dict, kind: str, M: int, L_avg: float):
+    """(bytes, flops) the method must move / compute in one call of `kind`."""
+    h, f, a = p["h"], p["ffn"], p["heads"]
+    d = h // a
+    wb = 0.5 + 4 / 64 if p["w_bits"] == 4 else 2.0
+    kvb = (d / 2 + 4 * d / 64) if p["kv_bits"] == 4 else 2 * d  # bytes per cached row
+    gemm = {"qkv": (3 * h, h, False), "out_proj": (h, h, True), "fc1": (f, h, False),
+            "fc2": (h, f, True)}
+    if kind in gemm:
+        n, k, res = gemm[kind]
+        byts = n * k * wb + M * k * 2 + M * n * 2 * (2 if res else 1) + n * 2
+        return byts, 2.0 * M * n * k
+    if kind == "attn_decode":
+        return M * a * L_avg * 2 * kvb + 2 * M * h * 2, 4.0 * M * L_avg * h
+    if kind == "kv_append":
+        return M * 2 * h * 2 + M * a * 2 * kvb, 0.0
+    if kind == "layernorm":
+        return M * h * 4 + 4 * h, 0.0
+    if kind == "lm_head":
+        return p["vocab"] * h * 2 + M * h * 2 + M * p["vocab"] * 4, 2.0 * M * p["vocab"] * h
+    if kind == "argmax":
+        return M * p["vocab"] * 4, 0.0
+    if kind == "embed":
+        return M * h * 6, 0.0
+    return 0.0, 0.0
+
+
+def roofline(p, kind, calls, ms_total, M, L_avg, peaks):
+    byts, flops = kernel_work(p, kind, M, L_avg)
+    t = ms_total / calls / 1e3
+    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops > 0 and flops / max(byts, 1.0) > ridge:
+        ach = flops / t / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        return {"kernel": kind, "bound": "tensor", "achieved": round(ach, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                "peak_note": f"{peaks['source']} dense bf16 sustained (fp16 nominal ratio 1:1)",
+                "algorithmic_per_launch": {"flops": flops, "bytes": byts}}
+    ach = byts / t / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"kernel": kind, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(ach / peak, 4), "peak_note": f"{peaks['source']} HBM copy",
+            "algorithmic_per_launch": {"flops": flops, "bytes": byts}}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """One layer of the workload on the CPU oracle: a decode step for b_o
+    sequences at the average KV length s + n/2 over a seeded cache."""
+
+    def __init__(self, p: dict, b_o: int):
+        from oracle import opt
+        self.opt = opt
+        self.p = p
+        self.b_o = b_o
+        self.cfg = opt.Config.from_preset(p)
+        seed = synth.config_seed(p)
+        self.W = opt.effective_layer(self.cfg, opt.raw_layer(self.cfg, seed, 0))
+        self.L = p["s"] + p["n"] // 2
+        self.cache = opt.KVCache(self.cfg, b_o, self.L + 1, self.cfg.kv_bits)
+        h = p["h"]
+        hist = synth.normal_f16(seed, synth.TID_TEST_BASE + 1, b_o * self.L * h, 1.0)
+        hist = hist.reshape(b_o, self.L, h)
+        self.cache.write("k", hist, 0)
+        self.cache.write("v", hist, 0)
+        self.t = synth.normal_f16(seed, synth.TID_TEST_BASE + 2, b_o * h, 1.0).reshape(b_o, h)
+        self.t = self.t.astype(np.float64)
+
+    def step(self) -> float:
+        t0 = time.perf_counter()
+        self.opt.layer_decode(self.cfg, self.W, self.t, self.cache, self.L)
+        return time.perf_counter() - t0
+
+    def tokens_per_s(self, seconds: float) -> float:
+        # one decode token of one sequence needs all l layers
+        return self.b_o / (seconds * self.p["layers"])
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 0) for i in threadpool_info()), default=0)
+        if n:
+            return int(n)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(p: dict, budget_s: float = 12.0):
+    t_setup = time.perf_counter()
+    smp = OracleSample(p, b_o=4)
+    setup = time.perf_counter() - t_setup
+    smp.step()  # warm
+    times = []
+    t_end = time.perf_counter() + budget_s
+    while time.perf_counter() < t_end or len(times) < 3:
+        times.append(smp.step())
+    t = statistics.median(times)
+    return {"value": round(smp.tokens_per_s(t), 4), "unit": "tokens/s", "cores": cpu_cores(),
+            "kind": "oracle",
+            "sample": (f"oracle (numpy float64) decode of layer 0 for {smp.b_o} sequences at KV "
+                       f"length {smp.L + 1}, {len(times)} repetitions, median {t * 1e3:.1f} ms, "
+                       f"extrapolated x{p['layers']} layers per token; setup {setup:.0f} s "
+                       "(weights drawn, quantized, dequantized on the host)")}
+
+
+def run_reference(args, p):
+    import torch.distributed as dist  # noqa: F401
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    smp = OracleSample(p, b_o=4)
+    for _ in range(args.warmup):
+        smp.step()
+    times = [smp.step() for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    v = smp.tokens_per_s(t)
+    line = {"metric": METRIC, "value": round(v, 4), "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.config, "global_batch": smp.b_o, "seq_len": p["s"],
+                       "gen_tokens": p["n"], "note": "one layer per step, extrapolated"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores(),
+                             "kind": "oracle",
+                             "sample": f"layer-0 decode of {smp.b_o} sequences at KV length "
+                                       f"{smp.L + 1} per step, x{p['layers']} layers"},
+            "e2e": {"value": round(v, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "decode tokens/s, OPT-30B-shape 4-bit W+KV; HBM GB/s & tensor util vs peak"
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_flexq(args, p):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    from quantized_opt_decode_b200 import build
+    build.build()
+    from quantized_opt_decode_b200 import flexq as fq
+    from quantized_opt_decode_b200.device_model import DeviceModel, workspace
+
+    b, s, n, gbs = p["b"], p["s"], p["n"], p["gpu_batch"]
+    stream = torch.cuda.Stream()
+    t_setup = time.perf_counter()
+    with torch.cuda.stream(stream):
+        dm = DeviceModel(p, b=b, max_len=s + n, stream=stream)
+        prompts = torch.empty(b, s, dtype=torch.int32, device="cuda")
+        fq.flexq_synth_tokens(prompts, b * s, synth.config_seed(p), synth.TID_PROMPT + 7919 * rank,
+                              p["vocab"], stream=stream)
+        out = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+        ws_n = fq.flexq_generate_workspace(dm.struct, b, s, gbs)
+        ws = workspace(ws_n)
+    stream.synchronize()
+    setup_s = time.perf_counter() - t_setup
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    # prefill column once (fills every layer's cache)
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    fq.flexq_generate_prefill(dm.struct, prompts, b, s, n, gbs, out, ws, ws_n, stream)
+    e1.record(stream)
+    stream.synchronize()
+    prefill_ms = e0.elapsed_time(e1)
+    fq.flexq_device_status(stream)
+
+    def step():
+        fq.flexq_generate_decode(dm.struct, b, s, n, gbs, out, ws, ws_n, stream)
+
+    for _ in range(args.warmup):
+        step()
+    stream.synchronize()
+    fq.flexq_device_status(stream)
+
+    with ClockSampler(local) as clk:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        l0 = fq.flexq_launch_count()
+        t0, t1 = ev(), ev()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        launches = fq.flexq_launch_count() - l0
+        if world > 1:
+            dist.barrier()
+    clocks = clk.summary()
+    ms = t0.elapsed_time(t1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    fq.flexq_device_status(stream)
+    value = world * b * (n - 1) / (ms / 1e3)
+
+    # per-kernel breakdown: one more decode phase with every kernel bracketed
+    fq.flexq_profile_start()
+    step()
+    prof = fq.flexq_profile_stop(stream)
+    peaks = load_peaks()
+    L_avg = s + n / 2.0
+    kernels = {}
+    total = sum(v[0] for v in prof.values())
+    for kind, (kms, calls) in prof.items():
+        if calls == 0:
+            continue
+        M = b if kind not in ("lm_head", "argmax", "embed") else b
+        rl = roofline(p, kind, calls, kms, gbs if kind in ("qkv", "out_proj", "fc1", "fc2",
+                                                            "attn_decode", "kv_append",
+                                                            "layernorm") else M, L_avg, peaks)
+        kernels[kind] = {"calls": calls, "ms": round(kms, 3), "share": round(kms / total, 4),
+                         "avg_us": round(kms / calls * 1e3, 2), "bound": rl["bound"],
+                         "achieved": rl["achieved"], "unit": rl["unit"], "frac": rl["frac"]}
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
+    rl = roofline(p, dom, prof[dom][1], prof[dom][0], gbs, L_avg, peaks)
+    rl["traffic"] = ncu_traffic(dom)
+    rl.pop("algorithmic_per_launch", None)
+
+    # end to end through flexq_generate: prompts from pinned host memory,
+    # tokens back to pinned host memory, all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        host_prompts = prompts.cpu().pin_memory()
+        host_out = torch.empty(b, n, dtype=torch.int32).pin_memory()
+        dev_prompts = torch.empty_like(prompts)
+
+        def e2e_step():
+            dev_prompts.copy_(host_prompts, non_blocking=True)
+            fq.flexq_generate(dm.struct, dev_prompts, b, s, n, gbs, out, ws, ws_n, None, stream)
+            host_out.copy_(out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+            stream.synchronize()
+            a0, a1 = ev(), ev()
+            a0.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            a1.record(stream)
+        stream.synchronize()
+        e_ms = a0.elapsed_time(a1) / args.e2e_steps
+        if world > 1:
+            tt = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": round(world * b * n / (e_ms / 1e3), 2), "unit": "tokens/s",
+               "h2d_bytes_per_step": b * s * 4, "d2h_bytes_per_step": b * n * 4,
+               "ms_per_step": round(e_ms, 2),
+               "what": "flexq_generate end to end (prompt upload, prefill column, n-1 decode "
+                       "columns, token download): generated tokens b*n per second"}
+        fq.flexq_device_status(stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(p)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic (seeded splitmix64 draws; weights ~N(0,0.02) quantized to 4-bit)",
+            "config": {"workload": args.config, "layers": p["layers"], "h": p["h"],
+                       "heads": p["heads"], "ffn": p["ffn"], "vocab": p["vocab"],
+                       "global_batch": b * world, "gpu_batch": gbs, "seq_len": s,
+                       "gen_tokens": n, "w_bits": p["w_bits"], "kv_bits": p["kv_bits"],
+                       "parallelism": f"replicas x{world}",
+                       "step": "decode phase: n-1 decode columns x all layers + LM head",
+                       "l2": "no flush: inputs far larger than L2 (weights + KV per step)"},
+            "roofline": rl,
+            "kernels": kernels,
+            "prefill": {"ms": round(prefill_ms, 2),
+                        "tokens_per_s": round(world * b * s / (prefill_ms / 1e3), 1)},
+            "gpu_launches": int(launches),
+            "gpu_launches_per_step": int(launches // max(1, args.steps)),
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "setup_s": round(setup_s, 1),
+            "kernel_sources": csrc_hash(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="flexq", choices=["flexq", "reference"])
+    ap.add_argument("--config", default="opt-30b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    p = dict(synth.CONFIGS[args.config])
+    if args.impl == "reference":
+        run_reference(args, p)
+    else:
+        run_flexq(args, p)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,317 @@
+/*
+ * flexq: group-wise 4-bit OPT-style decoding on one B200 (sm_100a).
+ *
+ * C ABI of libflexq.so.  The operations follow the FlexGen pages:
+ *   [WT]  "FlexGen: High-Throughput Generative Inference of Large Language
+ *         Models with a Single GPU" walk-through (qingweiji.github.io):
+ *         section "P/D阶段计算" (prefill and decode equations), section
+ *         "内存占用分析" (biases, LayerNorms, tied embedding, KV cache shape
+ *         [b, s, a, h/a] and peak size), section "Throughput And Latency"
+ *         (generation throughput b n / t), section "Search Space" (GPU batch,
+ *         block = GPU batch x GPU batches, column-wise zig-zag traversal).
+ *   [RPT] "FlexGen研究学术报告" (fmread.com), section 三(C): group-wise
+ *         asymmetric 4-bit quantization of weights and KV cache, groups of 64
+ *         contiguous elements, dequantized to FP16 before compute.
+ *   [SRV] survey notes (gumorming.cn), "Transformer-Styles LLMs" eqs. (1)-(3)
+ *         (multi-head attention) and the word + positional embedding.
+ *
+ * Conventions (all entry points):
+ * - Memory: the caller allocates every buffer; the library never allocates
+ *   or frees device memory.  Pointers named *_dev are device pointers, *_host
+ *   host pointers.  fp16 tensors are passed as void* and are row-major.
+ * - Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Calls enqueue work and return without synchronising, unless a
+ *   comment says otherwise.
+ * - Errors: argument errors are detected on the host before any launch and
+ *   return FLEXQ_ERR_INVALID (or FLEXQ_ERR_WORKSPACE for a short workspace);
+ *   a failed launch returns FLEXQ_ERR_CUDA.  flexq_last_error() returns the
+ *   calling thread's last message.  Kernels never trap: a device-side wait
+ *   that runs out, or a token id out of range, sets a device error word that
+ *   flexq_device_status() reports.
+ * - Aliasing: outputs never alias inputs unless stated.
+ * - Shapes: h % 128 == 0, ffn % 128 == 0, d = h / heads in {64, 128}; linear
+ *   weights are stored [N_out][K_in] (y = x W^T + b) with K_in % 64 == 0.
+ */
+#ifndef FLEXQ_H
+#define FLEXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FLEXQ_OK = 0,
+  FLEXQ_ERR_INVALID = 1,     /* bad argument (null pointer, shape, alignment) */
+  FLEXQ_ERR_CUDA = 2,        /* a CUDA call or kernel launch failed */
+  FLEXQ_ERR_WORKSPACE = 3,   /* workspace pointer null or too small */
+  FLEXQ_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up */
+  FLEXQ_ERR_UNSUPPORTED = 5, /* valid request this build does not handle */
+  FLEXQ_ERR_DEVICE = 6       /* a kernel reported a bad device-side input */
+} flexq_status;
+
+/* Message of the calling thread's last failed call ("" if none). */
+const char* flexq_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int flexq_version(void);
+
+/* Synchronises `stream`, then reads and clears the device error word:
+ * FLEXQ_OK, FLEXQ_ERR_TIMEOUT (a bounded wait ran out) or FLEXQ_ERR_DEVICE
+ * (e.g. a token id outside [0, vocab)). */
+flexq_status flexq_device_status(void* stream);
+
+/* Deadline, in nanoseconds of device time, of every bounded wait inside the
+ * kernels (default 2e9; 0 restores the default).  A test knob: a tiny value
+ * makes pipelined kernels give up and report FLEXQ_ERR_TIMEOUT. */
+flexq_status flexq_set_wait_limit_ns(uint64_t ns);
+
+/* ------------------------------------------------------------------------ */
+/* Seeded synthetic inputs (not part of the method: workload generation).     */
+/* Element i of stream (seed, tensor_id) is splitmix64's output function      */
+/* (Steele, Lea and Flood 2014) applied to key + 0x9E3779B97F4A7C15 * (i + 1),  */
+/* key = mix(seed * 0x9E3779B97F4A7C15 + tensor_id).                          */
+/* ------------------------------------------------------------------------ */
+
+/* out_dev: n fp16.  Element i (of start .. start+n-1) is
+ * fp16_rn(fp32(sum of the hash's four 16-bit fields - 131070) * c + mean)
+ * with c = fp32(sqrt(3) / 65536 * sigma): ~N(mean, sigma^2) bounded at
+ * 3.46 sigma. */
+flexq_status flexq_synth_normal_f16(void* out_dev, size_t n, uint64_t seed, uint64_t tensor_id,
+                                    size_t start, float sigma, float mean, void* stream);
+
+/* out_dev: n int32 ids, ((hash >> 32) * vocab) >> 32, uniform on [0, vocab). */
+flexq_status flexq_synth_tokens(int32_t* out_dev, size_t n, uint64_t seed, uint64_t tensor_id,
+                                size_t start, int32_t vocab, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Group-wise asymmetric 4-bit codec [RPT 三(C)].                              */
+/* ------------------------------------------------------------------------ */
+
+/* x_dev: n fp16 (n % 64 == 0, |x| <= 2^15, finite), groups = runs of 64
+ * contiguous elements.  Outputs: codes_dev n/2 bytes (byte j = code[2j] |
+ * code[2j+1] << 4), min_dev and scale_dev n/64 fp16 each.  Per group:
+ * scale = fp16_rn((max - min) / 15), min = fp16(min) (-0 stored as +0),
+ * code = clamp(rint((x - min) / scale), 0, 15) (0 when scale == 0), all in
+ * fp32 round-to-nearest-even without fused multiply-add: bit-exact by
+ * contract.  All pointers 16-byte aligned. */
+flexq_status flexq_quantize(const void* x_dev, size_t n, uint8_t* codes_dev, void* min_dev,
+                            void* scale_dev, void* stream);
+
+/* Inverse: out_dev n fp16, x_hat = fp16_rn(fp32(code * scale) + min). */
+flexq_status flexq_dequantize(const uint8_t* codes_dev, const void* min_dev,
+                              const void* scale_dev, size_t n, void* out_dev, void* stream);
+
+/* Bytes of a 4-bit weight [n_out][k_in] in the GEMM's tiled layout:
+ * ceil(n_out / 128) * (k_in / 64) tiles of 4608 bytes, each tile = 128 rows x
+ * 32 bytes of codes (nibble order within every 32-bit word: element e in
+ * nibble (e >> 1) + 4 (e & 1)) followed by 128 (min, scale) fp16 pairs;
+ * tiles ordered [row tile][k block]; rows past n_out are zero. */
+size_t flexq_packed_weight_bytes(int n_out, int k_in);
+
+/* Canonical codec output (codes [n_out][k_in/2], min/scale [n_out][k_in/64])
+ * -> tiled layout (a pure permutation; bit-exact). */
+flexq_status flexq_pack_weight_q4(const uint8_t* codes_dev, const void* min_dev,
+                                  const void* scale_dev, int n_out, int k_in, void* packed_dev,
+                                  void* stream);
+
+/* fp16 W [n_out][k_in] -> tiled 4-bit layout in one pass (same codes as
+ * flexq_quantize followed by flexq_pack_weight_q4). */
+flexq_status flexq_quantize_weight_q4(const void* w_dev, int n_out, int k_in, void* packed_dev,
+                                      void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Layer building blocks.                                                     */
+/* ------------------------------------------------------------------------ */
+
+/* Y[m][n] = epilogue(X[m][k] W^T): the linear layers of [WT] "P/D阶段计算".
+ * x_dev fp16 [m][ldx] (ldx % 8 == 0, 16-byte aligned); w_dev: packed 4-bit
+ * (w_bits = 4) or fp16 [n][k] (w_bits = 16, n may be any size).  epilogue
+ * flags: 1 = + bias[n], 2 = GELU (erf form) after the bias, 4 = + residual
+ * [m][ld_res] last, 8 = write fp32 (alone).  y_dev fp16 (or fp32) [m][ldy].
+ * ws: fp32 partial sums when K is split across CTAs; size from
+ * flexq_linear_workspace (0 means none needed). */
+size_t flexq_linear_workspace(int m, int n, int k, int w_bits);
+flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_bits, int m, int n,
+                          int k, const void* bias_dev, const void* residual_dev, int ld_res,
+                          int epilogue, void* y_dev, int ldy, void* ws_dev, size_t ws_bytes,
+                          int force_splits, void* stream);
+
+/* LayerNorm of rows [rows][h] (biased variance, fp32 statistics). */
+flexq_status flexq_layernorm(const void* x_dev, int ldx, const void* gamma_dev,
+                             const void* beta_dev, void* y_dev, int ldy, int rows, int h,
+                             float eps, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Model description.                                                         */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  int h;        /* hidden size, % 128 == 0 */
+  int heads;    /* attention heads; d = h / heads in {64, 128} */
+  int ffn;      /* MLP width (ih), % 128 == 0 */
+  int w_bits;   /* 4 (packed tiled weights) or 16 (fp16 [N_out][K_in]) */
+  int kv_bits;  /* 4 (group-wise codes) or 16 (fp16) */
+  float ln_eps; /* LayerNorm epsilon (1e-5) */
+} flexq_config;
+
+/* One decoder layer's parameters (device pointers).  Linear weights [N_out]
+ * [K_in]: w_qkv [3h][h] (rows: Q heads, then K heads, then V heads, head j
+ * at rows j*d .. j*d+d-1), w_o [h][h], w_fc1 [ffn][h], w_fc2 [h][ffn];
+ * packed per flexq_packed_weight_bytes when w_bits == 4.  Biases and
+ * LayerNorm parameters fp16: b_qkv [3h], b_o [h], b_fc1 [ffn], b_fc2 [h],
+ * ln*_g / ln*_b [h]. */
+typedef struct {
+  const void *w_qkv, *w_o, *w_fc1, *w_fc2;
+  const void *b_qkv, *b_o, *b_fc1, *b_fc2;
+  const void *ln1_g, *ln1_b, *ln2_g, *ln2_b;
+} flexq_layer;
+
+/* One layer's KV cache for b sequences, max_len slots each ([WT]
+ * "内存占用分析": K and V of shape [b, s, a, h/a], stored here head-major).
+ * kv_bits == 4: k, v = codes [b][heads][max_len][d/2] (canonical nibble
+ * order), k_meta, v_meta = (min, scale) fp16 pairs [b][heads][max_len][d/64].
+ * kv_bits == 16: k, v = fp16 [b][heads][max_len][d]; metas NULL.  A GPU batch
+ * of sequences i0.. is the same layout with pointers advanced by i0 rows of
+ * heads * max_len slots. */
+typedef struct {
+  void *k, *v, *k_meta, *v_meta;
+  int b, max_len;
+} flexq_kv;
+
+/* Bytes of K (codes or values) + V + their metadata for one layer. */
+size_t flexq_kv_bytes(const flexq_config* cfg, int b, int max_len);
+
+/* Quantize-on-append, the decode update x_K <- Concat(x_K, t W_K) (and V)
+ * of [WT] "P/D阶段计算", and the prefill's bulk write.  k_dev, v_dev: fp16
+ * rows [b * ntok][ld] (row i*ntok + t, head j at columns j*d ..) written to
+ * slots pos0 .. pos0+ntok-1.  In 4-bit mode each (sequence, head, token)
+ * row is quantized exactly as flexq_quantize would quantize it. */
+flexq_status flexq_kv_append(const flexq_config* cfg, const flexq_kv* kv, const void* k_dev,
+                             const void* v_dev, int ld, int b, int pos0, int ntok, void* stream);
+
+/* Decode attention: out[i][j*d ..] = softmax(q_ij K_ij^T / sqrt(d)) V_ij over
+ * slots 0..len-1 of the cache (dequantized in 4-bit mode).  q_dev fp16
+ * [b][ldq] (head j at columns j*d), out_dev fp16 [b][ldo]. */
+flexq_status flexq_attention_decode(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev,
+                                    int ldq, int b, int len, void* out_dev, int ldo, void* stream);
+
+/* Causal prefill attention on fp16 Q/K/V: qkv_dev [b*s][ldqkv] with Q, K, V
+ * at column offsets 0, h, 2h; out_dev [b*s][ldo]. */
+flexq_status flexq_attention_prefill(const flexq_config* cfg, const void* qkv_dev, int ldqkv,
+                                     int b, int s, void* out_dev, int ldo, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Layer steps ([WT] "P/D阶段计算", pre-LN OPT block).                          */
+/*   u = LN1(x); [Q|K|V] = u W_qkv^T + b_qkv; o = attention;                   */
+/*   x_out = o W_o^T + b_o + x; v = LN2(x_out);                                */
+/*   y = GELU(v W_1^T + b_1) W_2^T + b_2 + x_out.                              */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes for a prefill over `rows` = b*s tokens (mode 0) or a decode
+ * over `rows` = b sequences (mode 1). */
+size_t flexq_layer_workspace(const flexq_config* cfg, int rows, int mode);
+
+/* Prefill of one layer over b sequences of s tokens: x_dev, y_dev fp16
+ * [b*s][h] (distinct).  Writes cache slots 0..s-1 (quantized in 4-bit
+ * mode); attention uses the pass's own fp16 K/V. */
+flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* layer,
+                                 const void* x_dev, void* y_dev, const flexq_kv* kv, int b, int s,
+                                 void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Decode of one layer for the token at position pos of b sequences: t_dev,
+ * y_dev fp16 [b][h] (distinct).  Appends this token's K/V to slot pos, then
+ * attends over slots 0..pos read back from the cache. */
+flexq_status flexq_layer_decode(const flexq_config* cfg, const flexq_layer* layer,
+                                const void* t_dev, void* y_dev, const flexq_kv* kv, int b,
+                                int pos, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Generation over a block ([WT] "Search Space" and "Throughput And Latency"). */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  flexq_config cfg;
+  int layers;
+  int vocab;
+  int max_pos;                /* rows of pos_embed */
+  const flexq_layer* layer;   /* host array [layers] of device-pointer sets */
+  const flexq_kv* kv;         /* host array [layers]; each b x max_len >= s+n */
+  const void* embed;          /* fp16 E [vocab][h]; also the tied LM head */
+  const void* pos_embed;      /* fp16 P [max_pos][h] */
+  const void* lnf_g;          /* final LayerNorm, fp16 [h] */
+  const void* lnf_b;
+} flexq_model;
+
+typedef struct {
+  float prefill_ms; /* device time of embedding + prefill + first token */
+  float decode_ms;  /* device time of the n-1 decode steps */
+} flexq_timing;
+
+/* Workspace bytes for flexq_generate (and its two halves below). */
+size_t flexq_generate_workspace(const flexq_model* model, int b, int s, int gpu_batch);
+
+/* The prefill column of flexq_generate alone: embeds the prompts, runs every
+ * layer over every GPU batch (filling cache slots 0..s-1) and writes token 1
+ * to out_dev[i*n + 0]. */
+flexq_status flexq_generate_prefill(const flexq_model* model, const int32_t* prompt_dev, int b, int s,
+                                    int n, int gpu_batch, int32_t* out_dev, void* ws_dev,
+                                    size_t ws_bytes, void* stream);
+
+/* The n-1 decode columns of flexq_generate alone: column j reads token
+ * out_dev[i*n + j-1] at position s+j-1, appends its K/V to slot s+j-1 of every
+ * layer and writes out_dev[i*n + j].  Needs the caches a prefill over the same
+ * b sequences left (slots 0..s-1); re-running it rewrites slots s..s+n-2. */
+flexq_status flexq_generate_decode(const flexq_model* model, int b, int s, int n, int gpu_batch,
+                                   int32_t* out_dev, void* ws_dev, size_t ws_bytes, void* stream);
+
+/* Greedy generation for a block of b sequences (prompt length s, n output
+ * tokens) processed as GPU batches of gpu_batch sequences (b % gpu_batch ==
+ * 0).  Zig-zag order: for each token column, for each layer, for each GPU
+ * batch; the prefill column emits token 1 from the last prompt position, each
+ * of the n-1 decode columns emits one more (lowest index among equal
+ * logits).  prompt_dev int32 [b][s], out_dev int32 [b][n].  With timing !=
+ * NULL the call synchronises the stream and fills it. */
+flexq_status flexq_generate(const flexq_model* model, const int32_t* prompt_dev, int b, int s,
+                            int n, int gpu_batch, int32_t* out_dev, void* ws_dev, size_t ws_bytes,
+                            flexq_timing* timing, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Instrumentation (measurement only; not part of the method).                */
+/* ------------------------------------------------------------------------ */
+
+/* Number of kernels this library has launched in the process so far. */
+uint64_t flexq_launch_count(void);
+
+/* Kernel kinds reported by the profiler. */
+typedef enum {
+  FLEXQ_K_LAYERNORM = 0,
+  FLEXQ_K_QKV = 1,
+  FLEXQ_K_KV_APPEND = 2,
+  FLEXQ_K_ATTN_PREFILL = 3,
+  FLEXQ_K_ATTN_DECODE = 4,
+  FLEXQ_K_OUT_PROJ = 5,
+  FLEXQ_K_FC1 = 6,
+  FLEXQ_K_FC2 = 7,
+  FLEXQ_K_EMBED = 8,
+  FLEXQ_K_LM_HEAD = 9,
+  FLEXQ_K_ARGMAX = 10,
+  FLEXQ_K_COUNT = 11
+} flexq_kernel_kind;
+
+/* Between start and stop, every kernel the layer steps and the generator
+ * launch is bracketed by two CUDA events on its stream (adds a little time;
+ * one host thread at a time).  stop synchronises `stream` and writes, per
+ * kind, the summed device milliseconds and the number of bracketed calls
+ * (a linear layer's call may hold a K-split finishing kernel as well). */
+flexq_status flexq_profile_start(void);
+flexq_status flexq_profile_stop(void* stream, float* total_ms /* [FLEXQ_K_COUNT] */,
+                                int* calls /* [FLEXQ_K_COUNT] */);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLEXQ_H */

@@ -1,0 +1,96 @@
+// Internal launch interface between the C ABI (flexq.cu) and the kernels.
+// Every launcher enqueues on `stream` and returns the launch status.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace flexq {
+
+// Bytes of one packed 4-bit weight tile: 128 rows x 64 codes (4096 B) followed
+// by 128 (min, scale) fp16 pairs (512 B).  Tiles are stored [n_tile][k_block].
+constexpr int kTileRows = 128;
+constexpr int kGroup = 64;
+constexpr int kTileCodeBytes = kTileRows * kGroup / 2;
+constexpr int kTileMetaBytes = kTileRows * 4;
+constexpr int kTileBytes = kTileCodeBytes + kTileMetaBytes;
+
+struct Runtime {
+  uint64_t wait_limit_ns;  // deadline of every bounded device wait
+  uint32_t* err;           // device error word
+  int num_sms;
+};
+const Runtime& runtime();
+
+// Counts one kernel launch of this library and returns the launch status.
+cudaError_t launched();
+
+// synthetic inputs
+cudaError_t launch_synth_normal(__half* out, size_t n, uint64_t key, size_t start, float scale,
+                                float mean, cudaStream_t s);
+cudaError_t launch_synth_tokens(int32_t* out, size_t n, uint64_t key, size_t start, int vocab,
+                                cudaStream_t s);
+
+// codec
+cudaError_t launch_quantize(const __half* x, size_t n, uint8_t* codes, __half* mn, __half* sc,
+                            cudaStream_t s);
+cudaError_t launch_dequantize(const uint8_t* codes, const __half* mn, const __half* sc, size_t n,
+                              __half* out, cudaStream_t s);
+cudaError_t launch_pack_weight(const uint8_t* codes, const __half* mn, const __half* sc, int n_out,
+                               int k_in, uint8_t* packed, cudaStream_t s);
+cudaError_t launch_quantize_weight(const __half* w, int n_out, int k_in, uint8_t* packed,
+                                   cudaStream_t s);
+
+// KV cache append (quantize on append in 4-bit mode)
+struct KvView {
+  void* k;        // 4-bit: codes [b][a][L][d/2]; 16-bit: fp16 [b][a][L][d]
+  void* v;
+  void* k_meta;   // 4-bit: (min, scale) fp16 pairs [b][a][L][d/64]
+  void* v_meta;
+  int max_len;
+};
+cudaError_t launch_kv_append(const __half* k_src, const __half* v_src, int ld_src, int b, int ntok,
+                             int heads, int d, int kv_bits, const KvView& kv, int pos0,
+                             cudaStream_t s);
+
+// LayerNorm over rows of width h (fp16 in/out, fp32 statistics)
+cudaError_t launch_layernorm(const __half* x, int ldx, const __half* g, const __half* bta,
+                             __half* y, int ldy, int rows, int h, float eps, cudaStream_t s);
+
+// GEMM: Y[m][n] = epilogue(X[m][k] . W[n][k]^T)
+enum Epilogue : int {
+  EPI_BIAS = 1,       // + bias[n]
+  EPI_GELU = 2,       // GELU (exact erf form) after the bias
+  EPI_RESIDUAL = 4,   // + residual[m][n] last
+  EPI_F32_OUT = 8,    // write fp32 (no bias/act/residual allowed)
+};
+struct LinearArgs {
+  const __half* x; int ldx;       // activations [m][k]
+  const void* w; int w_bits;      // packed 4-bit tiles, or fp16 [n][k]
+  int m, n, k;
+  const __half* bias;
+  const __half* residual; int ld_res;
+  void* y; int ldy;
+  int epi;
+  int force_splits;               // 0 = automatic
+  int force_tok_tile;             // 0 = automatic
+};
+size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits);
+cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
+
+// attention
+cudaError_t launch_attn_decode(const __half* q, int ldq, const KvView& kv, int b, int heads, int d,
+                               int kv_bits, int len, __half* out, int ldo, cudaStream_t s);
+cudaError_t launch_attn_prefill(const __half* qkv, int ldqkv, int b, int seq, int heads, int d,
+                                __half* out, int ldo, cudaStream_t s);
+
+// embedding and greedy choice
+cudaError_t launch_embed(const int32_t* tok, int ld_tok, int b, int ntok, const __half* E, int vocab,
+                         const __half* P, int pos0, int h, __half* x, cudaStream_t s);
+cudaError_t launch_argmax(const float* logits, int rows, int vocab, int ld, int32_t* out,
+                          int ld_out, cudaStream_t s);
+
+}  // namespace flexq

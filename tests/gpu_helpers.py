@@ -1,0 +1,66 @@
+"""Helpers shared by the GPU tests: host<->device copies and seeded inputs.
+(Test infrastructure; the oracle side never sees anything the GPU computed.)"""
+import numpy as np
+import torch
+
+from quantized_opt_decode_b200 import build
+
+build.build()
+
+from quantized_opt_decode_b200 import flexq as fq  # noqa: E402
+
+DEV = "cuda"
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def to_host(t: torch.Tensor) -> np.ndarray:
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def f16_groups(rng, n_groups, extra=True):
+    """fp16 test data: groups of 64 at magnitudes from 1e-6 to 1e4, plus the
+    codec's special cases (constant, +-0, subnormal ramp, two-valued, the
+    input-range boundary)."""
+    mags = 10.0 ** rng.uniform(-6, 4, size=(n_groups, 1))
+    x = (rng.standard_normal((n_groups, 64)) * mags + rng.standard_normal((n_groups, 1)) * mags)
+    x = x.astype(np.float16)
+    if extra and n_groups >= 8:
+        x[0] = np.float16(0.75)
+        x[1] = np.array([-0.0, 0.0] * 32, np.float16)
+        x[2] = (np.arange(64) * 2.0 ** -24).astype(np.float16)
+        x[3] = np.array([0.3, -1.7] * 32, np.float16)
+        x[4] = np.linspace(-32768, 32768, 64).astype(np.float16)
+        x[5] = np.float16(-0.0)
+        x[6, :] = np.float16(1.0)
+        x[6, 17] = np.float16(1.0009765625)
+    return x.reshape(-1)
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    d = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (d if d > 0 else 1.0))
+
+
+def tiled_to_canonical(packed: np.ndarray, n_out: int, k_in: int):
+    """Reads the GEMM's tiled 4-bit layout (as include/flexq.h documents it)
+    back into canonical codes [n_out][k_in/2] and min/scale [n_out][k_in/64]."""
+    kb = k_in // 64
+    nt = (n_out + 127) // 128
+    tiles = packed.reshape(nt, kb, 4608)
+    codes = np.ascontiguousarray(tiles[:, :, :4096]).view(np.uint32).reshape(nt, kb, 128, 8)
+    meta = np.ascontiguousarray(tiles[:, :, 4096:]).view(np.float16).reshape(nt, kb, 128, 2)
+    q = np.zeros((nt, kb, 128, 8, 8), np.uint8)
+    for e in range(8):
+        pos = (e >> 1) + 4 * (e & 1)
+        q[..., e] = (codes >> np.uint32(4 * pos)) & np.uint32(0xF)
+    # q[nt, kb, row, word, e] -> element (word*8+e) of group kb of row nt*128+row
+    q = q.transpose(0, 2, 1, 3, 4).reshape(nt * 128, kb * 64)[:n_out]
+    can = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
+    meta = meta.transpose(0, 2, 1, 3).reshape(nt * 128, kb, 2)[:n_out]
+    return can, meta[..., 0].copy(), meta[..., 1].copy()

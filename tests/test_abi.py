@@ -1,0 +1,128 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/flexq.h declares, and rejects bad arguments on the host before
+any launch (no compute call is made here)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "flexq.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(flexq_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def fq():
+    from quantized_opt_decode_b200 import build
+    build.build()
+    from quantized_opt_decode_b200 import flexq
+    return flexq
+
+
+def test_header_declares_the_pages_entry_points():
+    names = declared_functions()
+    for must in ("flexq_quantize", "flexq_dequantize", "flexq_layer_prefill",
+                 "flexq_layer_decode", "flexq_kv_append", "flexq_generate"):
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(fq):
+    lib = C.CDLL(fq._LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(declared_functions()) == set(fq.EXPORTED)
+
+
+def test_version_and_empty_error(fq):
+    assert fq.flexq_version() == 100
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+def test_codec_rejects_ragged_length(fq):
+    lib = fq._lib
+    assert lib.flexq_quantize(None, 65, None, None, None, None) == 1
+    assert "multiple of 64" in fq.flexq_last_error()
+    assert lib.flexq_dequantize(None, None, None, 100, None, None) == 1
+
+
+def test_codec_rejects_null_and_misaligned(fq):
+    lib = fq._lib
+    assert lib.flexq_quantize(None, 64, None, None, None, None) == 1
+    assert lib.flexq_quantize(0x1001, 64, 0x2000, 0x3000, 0x4000, None) == 1
+    assert "aligned" in fq.flexq_last_error()
+
+
+def test_packed_weight_size(fq):
+    assert fq.flexq_packed_weight_bytes(256, 128) == 2 * 2 * 4608
+    assert fq.flexq_packed_weight_bytes(130, 64) == 2 * 1 * 4608
+    assert fq.flexq_packed_weight_bytes(128, 65) == 0
+
+
+def test_config_validation(fq):
+    bad = [dict(h=100, heads=1), dict(h=256, heads=3), dict(h=256, heads=1),
+           dict(h=256, heads=4, ffn=100), dict(h=256, heads=4, w_bits=8)]
+    for over in bad:
+        kw = dict(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=4, ln_eps=1e-5)
+        kw.update(over)
+        cfg = fq.flexq_config(**kw)
+        assert fq._lib.flexq_kv_bytes(C.byref(cfg), 1, 8) == 0
+        assert fq._lib.flexq_layer_workspace(C.byref(cfg), 4, 1) == 0
+
+
+def test_kv_bytes_closed_forms(fq):
+    """fp16: 2 (K and V) * 2 bytes * b * L * h; 4-bit: 0.5 byte per element
+    plus 4 bytes of (min, scale) per 64 elements."""
+    for bits in (16, 4):
+        cfg = fq.flexq_config(h=7168, heads=56, ffn=28672, w_bits=4, kv_bits=bits, ln_eps=1e-5)
+        b, L = 144, 544
+        n = fq.flexq_kv_bytes(cfg, b, L)
+        per_elem = 2.0 if bits == 16 else 0.5 + 4 / 64
+        assert n == int(2 * per_elem * b * L * 7168)
+
+
+def test_layer_rejects_bad_arguments(fq):
+    cfg = fq.flexq_config(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=4, ln_eps=1e-5)
+    layer = fq.flexq_layer()
+    kv = fq.flexq_kv(0x1000, 0x2000, 0x3000, 0x4000, 4, 40)
+    st = fq._lib.flexq_layer_decode(C.byref(cfg), C.byref(layer), 0x1000, 0x2000, C.byref(kv), 4,
+                                    3, None, 0, None)
+    assert st == 1 and "NULL" in fq.flexq_last_error()
+    st = fq._lib.flexq_layer_decode(C.byref(cfg), None, 0x1000, 0x2000, C.byref(kv), 4, 50, None,
+                                    0, None)
+    assert st == 1 and "pos" in fq.flexq_last_error()
+
+
+def test_layer_rejects_short_workspace(fq):
+    cfg = fq.flexq_config(h=256, heads=4, ffn=1024, w_bits=16, kv_bits=16, ln_eps=1e-5)
+    ptrs = [0x10000 * (i + 1) for i in range(12)]
+    layer = fq.flexq_layer(*ptrs)
+    kv = fq.flexq_kv(0x100000, 0x200000, None, None, 4, 40)
+    need = fq._lib.flexq_layer_workspace(C.byref(cfg), 4, 1)
+    assert need > 0
+    st = fq._lib.flexq_layer_decode(C.byref(cfg), C.byref(layer), 0x300000, 0x400000, C.byref(kv),
+                                    4, 3, 0x500000, need - 1, None)
+    assert st == 3
+
+
+def test_generate_rejects_indivisible_gpu_batch(fq):
+    cfg = fq.flexq_config(h=256, heads=4, ffn=1024, w_bits=16, kv_bits=16, ln_eps=1e-5)
+    ptrs = [0x10000 * (i + 1) for i in range(12)]
+    layer = (fq.flexq_layer * 1)(fq.flexq_layer(*ptrs))
+    kv = (fq.flexq_kv * 1)(fq.flexq_kv(0x100000, 0x200000, None, None, 4, 40))
+    m = fq.flexq_model(cfg, 1, 512, 40, layer, kv, 0x1000, 0x2000, 0x3000, 0x4000)
+    st = fq._lib.flexq_generate(C.byref(m), 0x5000, 4, 32, 8, 3, 0x6000, 0x7000, 1 << 30, None,
+                                None)
+    assert st == 1 and "gpu_batch" in fq.flexq_last_error()
+    # s + n - 1 = 41 positions exceed max_pos = 40
+    st = fq._lib.flexq_generate(C.byref(m), 0x5000, 4, 32, 10, 4, 0x6000, 0x7000, 1 << 30, None,
+                                None)
+    assert st == 1 and "max_pos" in fq.flexq_last_error()

@@ -1,0 +1,167 @@
+"""GPU parity of the layer building blocks against the oracle on the same
+seeded fp16 inputs: LayerNorm, the dequant-fused tcgen05 linear layers (4-bit
+and fp16 weights, every epilogue, split K), the quantize-on-append KV write
+(bit-exact), decode attention over the 4-bit / fp16 cache and causal prefill
+attention.  Floating-point tolerance: 2e-3 relative Frobenius error (the
+layer-output bar), far above fp16 output rounding (~3e-4) and far below any
+indexing or operand mistake."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+from oracle import opt, q64  # noqa: E402
+from gpu_helpers import fq, rel_fro, to_dev, to_host  # noqa: E402
+
+TOL = 2e-3
+EPI = fq
+
+
+@pytest.mark.parametrize("rows,h", [(1, 256), (5, 256), (300, 7168), (3, 12288), (64, 2048)])
+def test_layernorm(rows, h):
+    rng = np.random.default_rng(rows * h)
+    x = (rng.standard_normal((rows, h)) * 2 + 0.5).astype(np.float16)
+    g = (1 + 0.1 * rng.standard_normal(h)).astype(np.float16)
+    b = (0.1 * rng.standard_normal(h)).astype(np.float16)
+    y = torch.empty(rows, h, dtype=torch.float16, device="cuda")
+    fq.flexq_layernorm(to_dev(x), h, to_dev(g), to_dev(b), y, h, rows, h, 1e-5)
+    ref = opt.layernorm(x.astype(np.float64), g.astype(np.float64), b.astype(np.float64), 1e-5)
+    assert rel_fro(to_host(y), ref) < TOL
+
+
+def _linear_case(m, n, k, w_bits, epi, splits, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((m, k)).astype(np.float16)
+    w = (rng.standard_normal((n, k)) * 0.05).astype(np.float16)
+    bias = (rng.standard_normal(n) * 0.1).astype(np.float16)
+    res = rng.standard_normal((m, n)).astype(np.float16)
+    if w_bits == 4:
+        wd = torch.empty(fq.flexq_packed_weight_bytes(n, k), dtype=torch.uint8, device="cuda")
+        fq.flexq_quantize_weight_q4(to_dev(w), n, k, wd)
+        w_eff = q64.roundtrip(w).astype(np.float64)
+    else:
+        wd = to_dev(w)
+        w_eff = w.astype(np.float64)
+    f32 = epi == fq.EPI_F32_OUT
+    y = torch.empty(m, n, dtype=torch.float32 if f32 else torch.float16, device="cuda")
+    ws_bytes = max(m * n * 4, 1)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    fq.flexq_linear(to_dev(x), k, wd, w_bits, m, n, k, to_dev(bias), to_dev(res), n, epi, y, n,
+                    ws, ws_bytes, splits)
+    ref = x.astype(np.float64) @ w_eff.T
+    if epi & fq.EPI_BIAS:
+        ref = ref + bias.astype(np.float64)
+    if epi & fq.EPI_GELU:
+        ref = opt.gelu(ref)
+    if epi & fq.EPI_RESIDUAL:
+        ref = ref + res.astype(np.float64)
+    return to_host(y), ref
+
+
+LIN_CASES = [
+    # m, n, k, epilogue, forced K splits
+    (1, 128, 64, 1, 0),
+    (4, 384, 256, 1, 0),
+    (17, 256, 1024, 1 | 2, 0),
+    (144, 512, 512, 1 | 4, 0),
+    (144, 256, 2048, 1 | 4, 5),
+    (32, 128, 4096, 1, 0),
+    (256, 384, 384, 1 | 2, 0),
+    (300, 384, 320, 1, 0),
+    (600, 256, 128, 1 | 4, 0),
+    (1000, 640, 512, 1 | 2, 3),
+    (7, 200, 192, 8, 0),
+    (3, 130, 64, 8, 0),
+]
+
+
+@pytest.mark.parametrize("m,n,k,epi,splits", LIN_CASES)
+def test_linear_q4(m, n, k, epi, splits):
+    got, ref = _linear_case(m, n, k, 4, epi, splits, m * 7 + n + k)
+    assert rel_fro(got, ref) < TOL, rel_fro(got, ref)
+
+
+@pytest.mark.parametrize("m,n,k,epi,splits", LIN_CASES + [(5, 1000, 256, 8, 0), (64, 50272 // 8, 256, 8, 0)])
+def test_linear_f16(m, n, k, epi, splits):
+    got, ref = _linear_case(m, n, k, 16, epi, splits, m * 11 + n + k)
+    assert rel_fro(got, ref) < TOL, rel_fro(got, ref)
+
+
+def test_linear_split_k_matches_unsplit():
+    a, ref = _linear_case(144, 512, 2048, 4, 1, 1, 3)
+    b, _ = _linear_case(144, 512, 2048, 4, 1, 8, 3)
+    assert rel_fro(a, ref) < TOL and rel_fro(b, ref) < TOL and rel_fro(a, b) < 1e-3
+
+
+def _cfg(h, heads, kv_bits):
+    return fq.flexq_config(h=h, heads=heads, ffn=4 * h, w_bits=4, kv_bits=kv_bits, ln_eps=1e-5)
+
+
+def _dev_cache(cfg, b, max_len):
+    from quantized_opt_decode_b200.device_model import KVCache
+    return KVCache(cfg, b, max_len)
+
+
+@pytest.mark.parametrize("h,heads", [(256, 4), (512, 4)])
+def test_kv_append_bit_exact(h, heads):
+    """Each (sequence, head, token) row quantized exactly as the oracle does."""
+    cfg = _cfg(h, heads, 4)
+    b, ntok, L, pos0 = 3, 5, 12, 4
+    rng = np.random.default_rng(h)
+    ld = 3 * h
+    rows = rng.standard_normal((b * ntok, ld)).astype(np.float16)
+    dev = _dev_cache(cfg, b, L)
+    rd = to_dev(rows)
+    fq.flexq_kv_append(cfg, dev.struct, rd[:, h:], rd[:, 2 * h:], ld, b, pos0, ntok)
+    ocfg = opt.Config(layers=1, h=h, heads=heads, ffn=4 * h, vocab=8, w_bits=4, kv_bits=4)
+    oc = opt.KVCache(ocfg, b, L, 4)
+    oc.write("k", rows[:, h:2 * h].reshape(b, ntok, h), pos0)
+    oc.write("v", rows[:, 2 * h:].reshape(b, ntok, h), pos0)
+    d = h // heads
+    kc = to_host(dev.k).reshape(b, heads, L, d // 2)
+    km = to_host(dev.k_meta).reshape(b, heads, L, d // 64, 2)
+    vc = to_host(dev.v).reshape(b, heads, L, d // 2)
+    assert np.array_equal(kc, oc.t["k_codes"])
+    assert np.array_equal(vc, oc.t["v_codes"])
+    assert np.array_equal(km[..., 0].view(np.uint16), oc.t["k_min"].view(np.uint16))
+    assert np.array_equal(km[..., 1].view(np.uint16), oc.t["k_scale"].view(np.uint16))
+
+
+@pytest.mark.parametrize("h,heads,kv_bits,length", [(256, 4, 4, 1), (256, 4, 4, 37), (512, 4, 4, 545),
+                                                    (256, 4, 16, 33), (512, 4, 16, 300),
+                                                    (1024, 8, 4, 1030)])
+def test_attention_decode(h, heads, kv_bits, length):
+    cfg = _cfg(h, heads, kv_bits)
+    b, L = 3, length + 3
+    rng = np.random.default_rng(length + h)
+    hist = rng.standard_normal((b * length, 3 * h)).astype(np.float16)
+    dev = _dev_cache(cfg, b, L)
+    hd = to_dev(hist)
+    fq.flexq_kv_append(cfg, dev.struct, hd[:, h:], hd[:, 2 * h:], 3 * h, b, 0, length)
+    q = rng.standard_normal((b, 3 * h)).astype(np.float16)
+    out = torch.empty(b, h, dtype=torch.float16, device="cuda")
+    fq.flexq_attention_decode(cfg, dev.struct, to_dev(q), 3 * h, b, length, out, h)
+    ocfg = opt.Config(layers=1, h=h, heads=heads, ffn=4 * h, vocab=8, w_bits=4, kv_bits=kv_bits)
+    oc = opt.KVCache(ocfg, b, L, kv_bits)
+    oc.write("k", hist[:, h:2 * h].reshape(b, length, h), 0)
+    oc.write("v", hist[:, 2 * h:].reshape(b, length, h), 0)
+    qq = q[:, :h].astype(np.float64).reshape(b, heads, h // heads)
+    ref = opt.attention_single(qq, oc.read("k", length), oc.read("v", length)).reshape(b, h)
+    assert rel_fro(to_host(out), ref) < TOL
+
+
+@pytest.mark.parametrize("h,heads,b,s", [(256, 4, 2, 1), (256, 4, 3, 37), (512, 4, 2, 64),
+                                         (512, 4, 2, 130), (1024, 8, 1, 257)])
+def test_attention_prefill(h, heads, b, s):
+    cfg = _cfg(h, heads, 16)
+    rng = np.random.default_rng(s + h)
+    qkv = rng.standard_normal((b * s, 3 * h)).astype(np.float16)
+    out = torch.empty(b * s, h, dtype=torch.float16, device="cuda")
+    fq.flexq_attention_prefill(cfg, to_dev(qkv), 3 * h, b, s, out, h)
+    x = qkv.astype(np.float64).reshape(b, s, 3 * h)
+    Q, K, V = (opt.heads_split(x[..., i * h:(i + 1) * h], heads) for i in range(3))
+    ref = opt.heads_merge(opt.attention_causal(Q, K, V)).reshape(b * s, h)
+    assert rel_fro(to_host(out), ref) < TOL

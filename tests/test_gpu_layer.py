@@ -1,0 +1,151 @@
+"""GPU parity of whole layer steps and of generation against the oracle.
+
+Layer steps (prefill over b x s tokens, then decode of one token) on the tiny
+configuration and on a d = 128 variant, 4-bit and fp16 weights/KV: max relative
+Frobenius error 2e-3 on the layer output, and on the layer's residual branch
+(y - x) a bound of 2e-3 relative to the output norm as well.  Cached codes are
+compared element by element: the K/V rows come out of a GEMM on each side, so
+a value sitting on a rounding boundary may land one code apart; at least 99%
+must be identical and none may differ by more than one step.
+
+Generation: tokens are a greedy choice, several of which can be right when two
+logits tie within rounding, so each GPU token is checked against the oracle
+run teacher-forced on the GPU's own tokens: it must be the oracle's argmax or
+within 2e-3 * max|logit| of it."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+import synth  # noqa: E402
+from oracle import opt  # noqa: E402
+from gpu_helpers import fq, rel_fro, to_dev, to_host  # noqa: E402
+from quantized_opt_decode_b200.device_model import DeviceModel, workspace  # noqa: E402
+
+TOL = 2e-3
+
+
+def _preset(name, **over):
+    p = dict(synth.CONFIGS[name])
+    p.update(over)
+    return p
+
+
+def _layer_roundtrip(p, b, s):
+    """Runs prefill then one decode through layer 0 on both sides."""
+    dm = DeviceModel(p, b=b, max_len=s + 4, layers=1)
+    cfg = opt.Config.from_preset(p)
+    seed = synth.config_seed(p)
+    W = opt.effective_layer(cfg, opt.raw_layer(cfg, seed, 0))
+    rng = np.random.default_rng(b * s + p["h"])
+    x = rng.standard_normal((b, s, p["h"])).astype(np.float16)
+    t = rng.standard_normal((b, p["h"])).astype(np.float16)
+    h = p["h"]
+    ws_n = max(fq.flexq_layer_workspace(dm.cfg, b * s, 0), fq.flexq_layer_workspace(dm.cfg, b, 1))
+    ws = workspace(ws_n)
+    xd = to_dev(x.reshape(b * s, h))
+    yd = torch.empty_like(xd)
+    L, kv = dm.layers[0].struct, dm.kv[0].struct
+    fq.flexq_layer_prefill(dm.cfg, L, xd, yd, kv, b, s, ws, ws_n)
+    td = to_dev(t)
+    t2 = torch.empty_like(td)
+    fq.flexq_layer_decode(dm.cfg, L, td, t2, kv, b, s, ws, ws_n)
+    fq.flexq_device_status()
+    y_ref, K16, V16 = opt.layer_prefill(cfg, W, x.astype(np.float64))
+    cache = opt.KVCache(cfg, b, s + 4, cfg.kv_bits)
+    cache.write("k", K16, 0)
+    cache.write("v", V16, 0)
+    t_ref = opt.layer_decode(cfg, W, t.astype(np.float64), cache, s)
+    return dm, (to_host(yd).reshape(b, s, h), y_ref, x), (to_host(t2), t_ref, t), cache
+
+
+def _check_out(got, ref, x):
+    assert rel_fro(got, ref) < TOL, rel_fro(got, ref)
+    branch = np.linalg.norm(got.astype(np.float64) - ref) / np.linalg.norm(ref - x.astype(np.float64))
+    assert branch < 1e-2, branch  # error relative to the layer's own contribution
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", {}),
+    ("tiny16", {}),
+    ("tiny", dict(h=512, heads=4, ffn=2048)),      # d = 128
+    ("tiny16", dict(h=512, heads=4, ffn=2048)),
+])
+def test_layer_prefill_and_decode(name, over):
+    p = _preset(name, **over)
+    dm, (y, y_ref, x), (t2, t_ref, t), cache = _layer_roundtrip(p, b=4, s=32)
+    _check_out(y, y_ref, x)
+    _check_out(t2, t_ref, t)
+    # cached K: element-wise comparison of codes (or fp16 values)
+    b, s, a, d = 4, 32, p["heads"], p["h"] // p["heads"]
+    if p["kv_bits"] == 4:
+        kc = to_host(dm.kv[0].k).reshape(b, a, s + 4, d // 2)
+        got = np.stack([kc & 15, kc >> 4], -1).astype(int)
+        oc = cache.t["k_codes"]
+        want = np.stack([oc & 15, oc >> 4], -1).astype(int)
+        diff = np.abs(got[:, :, :s + 1] - want[:, :, :s + 1])
+        assert diff.max() <= 1 and (diff == 0).mean() > 0.99
+    else:
+        kc = to_host(dm.kv[0].k).reshape(b, a, s + 4, d).astype(np.float64)
+        assert rel_fro(kc[:, :, :s + 1], cache.t["k"][:, :, :s + 1].astype(np.float64)) < TOL
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny16"])
+def test_generate_tokens_valid_under_oracle(name):
+    p = _preset(name)
+    b, s, n = p["b"], p["s"], p["n"]
+    dm = DeviceModel(p, b=b, max_len=s + n)
+    seed = synth.config_seed(p)
+    prompts = synth.tokens(seed, synth.TID_PROMPT, b * s, p["vocab"]).reshape(b, s)
+    out = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+    ws_n = fq.flexq_generate_workspace(dm.struct, b, s, p["gpu_batch"])
+    ws = workspace(ws_n)
+    timing = fq.flexq_timing()
+    fq.flexq_generate(dm.struct, to_dev(prompts), b, s, n, p["gpu_batch"], out, ws, ws_n, timing)
+    fq.flexq_device_status()
+    toks = to_host(out)
+    m = opt.build_model(opt.Config.from_preset(p), seed, s + n)
+    own, _ = opt.generate(m, prompts, n)
+    _, logits = opt.generate(m, prompts, n, forced=toks)
+    for j in range(n):
+        for i in range(b):
+            lg = logits[j, i]
+            assert lg[toks[i, j]] >= lg.max() - 2e-3 * np.abs(lg).max(), (i, j)
+    assert (toks == own).mean() > 0.5
+    assert timing.prefill_ms > 0 and timing.decode_ms > 0
+
+
+def test_block_schedule_gpu_batches_agree():
+    """The zig-zag block order with GPU batches of b, b/2 and b/4 sequences
+    produces the same tokens (sequences are independent)."""
+    p = _preset("tiny", b=8)
+    b, s, n = 8, p["s"], 6
+    dm = DeviceModel(p, b=b, max_len=s + n)
+    seed = synth.config_seed(p)
+    prompts = to_dev(synth.tokens(seed, synth.TID_PROMPT, b * s, p["vocab"]).reshape(b, s))
+    results = []
+    for gbs in (8, 4, 2):
+        out = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+        ws_n = fq.flexq_generate_workspace(dm.struct, b, s, gbs)
+        ws = workspace(ws_n)
+        fq.flexq_generate(dm.struct, prompts, b, s, n, gbs, out, ws, ws_n)
+        results.append(to_host(out))
+    assert np.array_equal(results[0], results[1]) and np.array_equal(results[0], results[2])
+
+
+def test_sequence_subset_matches_block():
+    """A GPU batch run alone yields the tokens it yields inside the block."""
+    p = _preset("tiny", b=4)
+    b, s, n = 4, p["s"], 5
+    dm = DeviceModel(p, b=b, max_len=s + n)
+    seed = synth.config_seed(p)
+    pr = synth.tokens(seed, synth.TID_PROMPT, b * s, p["vocab"]).reshape(b, s)
+    out = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+    ws_n = fq.flexq_generate_workspace(dm.struct, b, s, b)
+    ws = workspace(ws_n)
+    fq.flexq_generate(dm.struct, to_dev(pr), b, s, n, b, out, ws, ws_n)
+    full = to_host(out)
+    out2 = torch.zeros(2, n, dtype=torch.int32, device="cuda")
+    fq.flexq_generate(dm.struct, to_dev(pr[1:3]), 2, s, n, 2, out2, ws, ws_n)
+    assert np.array_equal(to_host(out2), full[1:3])
