@@ -139,6 +139,24 @@ flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_b
                           int epilogue, void* y_dev, int ldy, void* ws_dev, size_t ws_bytes,
                           int force_splits, void* stream);
 
+/* flexq_linear for callers that cannot allocate device memory.  The pages
+ * have no counterpart: this is a library-service entry point.  A caller such
+ * as a plug-in that a host framework hands only its input and output buffers
+ * (the framework's pool owning the rest of device memory), or a loop that
+ * must not pay for cudaMalloc/cudaFree, has no workspace to offer; here the
+ * K-split partial sums live in an 8 MiB array compiled into the library
+ * (reserved on every GPU that loads it until exit).  Arguments and results
+ * as flexq_linear, without ws.  Limit: when K is split, m * n <= 2,097,152;
+ * larger requests return FLEXQ_ERR_INVALID without launching.  The first
+ * call on a device looks up the array's address for that device: make it
+ * before any stream capture.  All calls share the array (each clears what it
+ * uses first); calls that overlap on the GPU race on it, so serialise them.
+ * Allocates nothing. */
+flexq_status flexq_linear_static_scratch(const void* x_dev, int ldx, const void* w_dev, int w_bits,
+                                         int m, int n, int k, const void* bias_dev,
+                                         const void* residual_dev, int ld_res, int epilogue,
+                                         void* y_dev, int ldy, int force_splits, void* stream);
+
 /* LayerNorm of rows [rows][h] (biased variance, fp32 statistics). */
 flexq_status flexq_layernorm(const void* x_dev, int ldx, const void* gamma_dev,
                              const void* beta_dev, void* y_dev, int ldy, int rows, int h,

@@ -286,6 +286,8 @@ const Runtime& runtime() {
 
 uint32_t* device_error_word() { return runtime().err; }
 
+void set_last_error(const char* msg) { g_last_error = msg; }
+
 cudaError_t launched() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError();

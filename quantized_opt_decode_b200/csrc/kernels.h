@@ -28,6 +28,9 @@ const Runtime& runtime();
 // Counts one kernel launch of this library and returns the launch status.
 cudaError_t launched();
 
+// Sets the calling thread's message returned by flexq_last_error().
+void set_last_error(const char* msg);
+
 // synthetic inputs
 cudaError_t launch_synth_normal(__half* out, size_t n, uint64_t key, size_t start, float scale,
                                 float mean, cudaStream_t s);

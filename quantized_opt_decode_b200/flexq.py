@@ -83,6 +83,8 @@ _SIGS = {
     "flexq_linear_workspace": ([C.c_int, C.c_int, C.c_int, C.c_int], C.c_size_t),
     "flexq_linear": ([VP, C.c_int, VP, C.c_int, C.c_int, C.c_int, C.c_int, VP, VP, C.c_int,
                       C.c_int, VP, C.c_int, VP, C.c_size_t, C.c_int, VP], C.c_int),
+    "flexq_linear_static_scratch": ([VP, C.c_int, VP, C.c_int, C.c_int, C.c_int, C.c_int, VP, VP,
+                                     C.c_int, C.c_int, VP, C.c_int, C.c_int, VP], C.c_int),
     "flexq_layernorm": ([VP, C.c_int, VP, VP, VP, C.c_int, C.c_int, C.c_int, C.c_float, VP],
                         C.c_int),
     "flexq_kv_bytes": ([_CFG, C.c_int, C.c_int], C.c_size_t),
@@ -191,6 +193,13 @@ def flexq_linear(x, ldx, w, w_bits, m, n, k, bias, residual, ld_res, epilogue, y
                  ws=None, ws_bytes=0, force_splits=0, stream=None):
     _check(_lib.flexq_linear(_p(x), ldx, _p(w), w_bits, m, n, k, _p(bias), _p(residual), ld_res,
                              epilogue, _p(y), ldy, _p(ws), ws_bytes, force_splits, _s(stream)))
+
+
+def flexq_linear_static_scratch(x, ldx, w, w_bits, m, n, k, bias, residual, ld_res, epilogue, y,
+                                ldy, force_splits=0, stream=None):
+    _check(_lib.flexq_linear_static_scratch(_p(x), ldx, _p(w), w_bits, m, n, k, _p(bias),
+                                            _p(residual), ld_res, epilogue, _p(y), ldy,
+                                            force_splits, _s(stream)))
 
 
 def flexq_layernorm(x, ldx, gamma, beta, y, ldy, rows, h, eps=1e-5, stream=None):

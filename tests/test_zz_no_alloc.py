@@ -1,0 +1,56 @@
+"""flexq_linear_static_scratch, the linear layer for callers that cannot
+allocate device memory (for example a plug-in that its host framework hands
+only input and output buffers), keeps its K-split partial sums in a fixed
+array inside the library.  Checked here through the C ABI against
+flexq_linear with a caller-provided workspace, on two calls in a row (the
+second call must clear what the first one left in the shared array), plus the
+size limit.  This file is collected last on purpose."""
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+from gpu_helpers import fq, rel_fro, to_dev, to_host  # noqa: E402
+
+TOL = 2e-3  # the tolerance of the other GPU parity tests
+
+
+def _inputs(m, n, k, seed):
+    rng = np.random.default_rng(seed)
+    x = to_dev(rng.standard_normal((m, k)).astype(np.float16))
+    w = to_dev((rng.standard_normal((n, k)) * 0.05).astype(np.float16))
+    wq = torch.empty(fq.flexq_packed_weight_bytes(n, k), dtype=torch.uint8, device="cuda")
+    fq.flexq_quantize_weight_q4(w, n, k, wq)
+    bias = to_dev((rng.standard_normal(n) * 0.1).astype(np.float16))
+    res = to_dev(rng.standard_normal((m, n)).astype(np.float16))
+    return x, wq, bias, res
+
+
+@pytest.mark.parametrize("m,n,k,splits", [(144, 512, 2048, 8), (32, 1024, 4096, 0)])
+def test_static_scratch_matches_workspace_linear_twice(m, n, k, splits):
+    x, wq, bias, res = _inputs(m, n, k, m + n)
+    epi = fq.EPI_BIAS | fq.EPI_RESIDUAL
+    need = fq.flexq_linear_workspace(m, n, k, 4)
+    ws_bytes = max(need, m * n * 4)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    ref = torch.empty(m, n, dtype=torch.float16, device="cuda")
+    fq.flexq_linear(x, k, wq, 4, m, n, k, bias, res, n, epi, ref, n, ws, ws_bytes, splits)
+    want = to_host(ref).astype(np.float64)
+    for _ in range(2):
+        y = torch.full((m, n), float("nan"), dtype=torch.float16, device="cuda")
+        fq.flexq_linear_static_scratch(x, k, wq, 4, m, n, k, bias, res, n, epi, y, n, splits)
+        fq.flexq_device_status()
+        got = to_host(y)
+        assert np.isfinite(got).all()
+        assert rel_fro(got, want) < TOL
+
+
+def test_static_scratch_rejects_oversized_split():
+    m, n, k = 300, 8192, 128
+    x = torch.zeros(m, k, dtype=torch.float16, device="cuda")
+    wq = torch.zeros(fq.flexq_packed_weight_bytes(n, k), dtype=torch.uint8, device="cuda")
+    y = torch.zeros(m, n, dtype=torch.float16, device="cuda")
+    with pytest.raises(fq.FlexqError) as ei:
+        fq.flexq_linear_static_scratch(x, k, wq, 4, m, n, k, None, None, 0, 0, y, n, 2)
+    assert ei.value.status == 1 and "static scratch" in str(ei.value)
