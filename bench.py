@@ -343,11 +343,13 @@ def run_flexq(args, p):
         torch.cuda.synchronize()
         l0 = fq.flexq_launch_count()
         t0, t1 = ev(), ev()
+        torch.cuda.nvtx.range_push("timed")
         t0.record(stream)
         for _ in range(args.steps):
             step()
         t1.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
         launches = fq.flexq_launch_count() - l0
         if world > 1:
             dist.barrier()
