@@ -131,9 +131,13 @@ flexq_status flexq_quantize_weight_q4(const void* w_dev, int n_out, int k_in, vo
  * (w_bits = 4) or fp16 [n][k] (w_bits = 16, n may be any size).  epilogue
  * flags: 1 = + bias[n], 2 = GELU (erf form) after the bias, 4 = + residual
  * [m][ld_res] last, 8 = write fp32 (alone).  y_dev fp16 (or fp32) [m][ldy].
- * ws: fp32 partial sums when K is split across CTAs; size from
- * flexq_linear_workspace (0 means none needed). */
-size_t flexq_linear_workspace(int m, int n, int k, int w_bits);
+ * ws: fp32 partial output tiles when K is shared out across CTAs (small
+ * grids) plus one counter per tile; size from flexq_linear_workspace with the
+ * same force_splits (0 means none needed).  force_splits = 0 lets the library
+ * choose (whole tiles per SM when there are many, equal shares of all
+ * k-blocks per SM when there are few); s > 1 cuts every tile's K into s parts
+ * (tests); 1 forbids splitting K. */
+size_t flexq_linear_workspace(int m, int n, int k, int w_bits, int force_splits);
 flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_bits, int m, int n,
                           int k, const void* bias_dev, const void* residual_dev, int ld_res,
                           int epilogue, void* y_dev, int ldy, void* ws_dev, size_t ws_bytes,
@@ -146,7 +150,8 @@ flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_b
  * must not pay for cudaMalloc/cudaFree, has no workspace to offer; here the
  * K-split partial sums live in an 8 MiB array compiled into the library
  * (reserved on every GPU that loads it until exit).  Arguments and results
- * as flexq_linear, without ws.  Limit: when K is split, m * n <= 2,097,152;
+ * as flexq_linear, without ws.  Limit: the K-split scratch the shape needs
+ * (flexq_linear_workspace with the same force_splits) must fit in 8 MiB;
  * larger requests return FLEXQ_ERR_INVALID without launching.  The first
  * call on a device looks up the array's address for that device: make it
  * before any stream capture.  All calls share the array (each clears what it
@@ -189,11 +194,14 @@ typedef struct {
 
 /* One layer's KV cache for b sequences, max_len slots each ([WT]
  * "内存占用分析": K and V of shape [b, s, a, h/a], stored here head-major).
- * kv_bits == 4: k, v = codes [b][heads][max_len][d/2] (canonical nibble
- * order), k_meta, v_meta = (min, scale) fp16 pairs [b][heads][max_len][d/64].
- * kv_bits == 16: k, v = fp16 [b][heads][max_len][d]; metas NULL.  A GPU batch
- * of sequences i0.. is the same layout with pointers advanced by i0 rows of
- * heads * max_len slots. */
+ * kv_bits == 4: k = codes [b][heads][max_len][d/2] (canonical nibble order);
+ * v = codes in 32-bit words [b][heads][L8/8][d] with L8 = max_len rounded up
+ * to a multiple of 8, token-interleaved: nibble k (bits 4k..4k+3) of word
+ * (block, e) is the code of token 8*block + k at dimension e; k_meta, v_meta
+ * = (min, scale) fp16 pairs [b][heads][max_len][d/64].  kv_bits == 16: k, v =
+ * fp16 [b][heads][max_len][d]; metas NULL.  A GPU batch of sequences i0.. is
+ * the same layout with pointers advanced by i0 rows of heads * max_len slots
+ * (heads * L8 for 4-bit V). */
 typedef struct {
   void *k, *v, *k_meta, *v_meta;
   int b, max_len;

@@ -146,7 +146,8 @@ KvView view_of(const flexq_config* c, const flexq_kv* kv, int seq0) {
   v.max_len = kv->max_len;
   if (c->kv_bits == 4) {
     v.k = static_cast<uint8_t*>(kv->k) + slots * (d / 2);
-    v.v = static_cast<uint8_t*>(kv->v) + slots * (d / 2);
+    v.v = static_cast<uint8_t*>(kv->v) +
+          static_cast<size_t>(seq0) * c->heads * kv_pad_len(kv->max_len) * (d / 2);
     v.k_meta = static_cast<uint8_t*>(kv->k_meta) + slots * (d / 64) * 4;
     v.v_meta = static_cast<uint8_t*>(kv->v_meta) + slots * (d / 64) * 4;
   } else {
@@ -401,9 +402,9 @@ flexq_status flexq_quantize_weight_q4(const void* w_dev, int n_out, int k_in, vo
 }
 
 // --- building blocks -----------------------------------------------------------
-size_t flexq_linear_workspace(int m, int n, int k, int w_bits) {
-  if (m <= 0 || n <= 0 || k <= 0 || k % 64) return 0;
-  return linear_workspace_bytes(m, n, k, w_bits, 0);
+size_t flexq_linear_workspace(int m, int n, int k, int w_bits, int force_splits) {
+  if (m <= 0 || n <= 0 || k <= 0 || k % 64 || force_splits < 0) return 0;
+  return linear_workspace_bytes(m, n, k, w_bits, force_splits);
 }
 
 flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_bits, int m, int n, int k,
@@ -463,7 +464,8 @@ size_t flexq_kv_bytes(const flexq_config* cfg, int b, int max_len) {
   if (check_config(cfg) != FLEXQ_OK || b <= 0 || max_len <= 0) return 0;
   const size_t elems = static_cast<size_t>(b) * max_len * cfg->h;  // per K or V
   if (cfg->kv_bits == 16) return 2 * elems * 2;
-  return 2 * (elems / 2 + elems / 64 * 4);
+  const size_t v_elems = static_cast<size_t>(b) * kv_pad_len(max_len) * cfg->h;  // whole 8-token blocks
+  return elems / 2 + v_elems / 2 + 2 * (elems / 64 * 4);
 }
 
 flexq_status flexq_kv_append(const flexq_config* cfg, const flexq_kv* kv, const void* k_dev, const void* v_dev,

@@ -9,22 +9,28 @@
 // walk-through (section "P/D阶段计算"), with the [h] / [ih] biases of section
 // "内存占用分析" fused into the epilogue.
 //
-// Design (one CTA = 128 output features x up to 256 tokens; the weight is the
-// MMA's A operand so that small decode batches become the MMA's N):
-//   warp 0      TMA producer: one cp.async.bulk of the packed 4-bit tile
-//               (codes + min/scale, 4608 contiguous bytes) and one tiled
-//               cp.async.bulk.tensor of the fp16 activations per 64-wide
-//               k-block, completion counted on an mbarrier;
-//   warps 2-9   dequantize: (code | 0x6400) is the fp16 value 1024 + code, one
-//               half2 subtract and one half2 fused multiply-add give
-//               code * scale + min rounded once to fp16, written straight into
-//               the 128-byte-swizzled K-major layout the tensor core reads;
-//   warp 1      allocates TMEM and, from one thread, issues
-//               tcgen05.mma.kind::f16 (M=128, N=tokens, K=16) x 4 per k-block,
-//               freeing each stage with tcgen05.commit;
-//   warps 2-9   epilogue: tcgen05.ld of the fp32 accumulator, + bias, GELU,
-//               + residual, fp16 store (or fp32 atomic partial sums when K is
-//               split across CTAs to fill the 148 SMs).
+// One output tile = 128 features x up to 256 tokens; the weight is the MMA's A
+// operand, so a small decode batch becomes the MMA's N.  A persistent CTA per
+// SM walks a list of (tile, k-block range) segments:
+//   warp 0      TMA producer: per 64-wide k-block one cp.async.bulk of the
+//               packed 4-bit chunk (codes + min/scale, 4608 contiguous bytes)
+//               or a tiled fp16 weight box, plus one 128-byte-swizzled
+//               cp.async.bulk.tensor of the activations, into a deep ring;
+//   warps 2-9   dequantize the chunk into a short ring of fp16 A tiles in the
+//               UMMA K-major SW128 layout ((code | 0x6400) is the fp16 value
+//               1024 + code; one half2 subtract and one half2 fused
+//               multiply-add give code * scale + min rounded once);
+//   warp 1      owns TMEM (two accumulator buffers) and, from one thread,
+//               issues tcgen05.mma.kind::f16 (M=128, N=tokens, K=16) x 4 per
+//               k-block, releasing ring slots with tcgen05.commit;
+//   warps 10-13 epilogue: tcgen05.ld, + bias, GELU, + residual, fp16 or fp32
+//               store; overlaps the next segment's main loop.
+// Scheduling: whole tiles round-robin over the SMs when there are many; when
+// the grid is small (decode), each SM takes an equal share of all k-blocks
+// (stream-K), so tiles may be split across CTAs.  A partial tile is written
+// to a per-contributor fp32 slot; the contributor that arrives last (an atomic
+// counter per tile) sums the slots in contributor order and applies the
+// epilogue, so results do not depend on timing.
 // Every mbarrier wait is bounded; on expiry the CTA records an error code in
 // the device error word and unwinds (no trap).
 #include <math.h>
@@ -37,21 +43,39 @@
 namespace flexq {
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kConsumers = 256;
+constexpr int kThreads = 448;
+constexpr int kDequantThreads = 256;
+constexpr int kEpiThreads = 128;
+constexpr int kEpiWarp0 = 10;
 constexpr int kATileBytes = 128 * 64 * 2;
 constexpr int kRawBytes = 5120;  // kTileBytes rounded up to keep 1 KB alignment
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kBarrierBytes = 256;
+constexpr int kBarrierBytes = 512;
+constexpr int kEpiStageBytes = 4 * 16 * 33 * 4;  // per epilogue warp: 16 tokens x 33 floats
+constexpr int kMaxLoadStages = 16;
+constexpr int kMinItersPerCta = 8;
+constexpr int kMaxContrib = 64;
+
+enum SchedMode : int { SCHED_TILES = 0, SCHED_STREAMK = 1, SCHED_SPLITS = 2 };
+
+struct Sched {
+  int mode;
+  int grid;
+  int tiles;        // n_tiles * tok_tiles
+  int n_tiles;
+  int kb_total;
+  long long iters;  // tiles * kb_total
+  int splits, per;  // SCHED_SPLITS
+};
 
 struct GemmParams {
   const uint8_t* wq;
   int m, n, k;
-  int kb_total, kb_per_split;
   int tok_tile;
-  int stages;
-  uint32_t stage_bytes;
-  uint32_t tmem_cols;
+  int load_stages, a_stages;
+  uint32_t load_stage_bytes;
+  uint32_t tmem_cols;  // per accumulator buffer
+  Sched sc;
   const __half* bias;
   const __half* residual;
   int ld_res;
@@ -60,10 +84,77 @@ struct GemmParams {
   float* yf;
   int ldyf;
   int epi;
-  int splitk;
+  float* partials;  // [slot][tok_tile][128]
+  int* counters;    // [tiles]
   uint64_t wait_ns;
   uint32_t* err;
 };
+
+struct Seg {
+  int tile, kb0, kb1;
+  bool full;
+  int slot;
+};
+
+// Position and phase parity in a ring of mbarrier-guarded slots, advanced
+// without divisions (the role threads are latency-bound scalar loops).
+struct Ring {
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
+__device__ __forceinline__ long long sk_start(const Sched& s, int c) {
+  return static_cast<long long>(c) * s.iters / s.grid;
+}
+
+// Segment q of CTA c; false when the CTA has no more work.
+__device__ __forceinline__ bool get_seg(const Sched& s, int c, int q, Seg& g) {
+  if (s.mode == SCHED_TILES) {
+    const long long t = c + static_cast<long long>(q) * s.grid;
+    if (t >= s.tiles) return false;
+    g.tile = static_cast<int>(t);
+    g.kb0 = 0;
+    g.kb1 = s.kb_total;
+    g.full = true;
+    g.slot = -1;
+    return true;
+  }
+  if (s.mode == SCHED_SPLITS) {
+    if (q > 0) return false;
+    g.tile = c / s.splits;
+    const int part = c % s.splits;
+    g.kb0 = part * s.per;
+    g.kb1 = min(s.kb_total, g.kb0 + s.per);
+    g.full = s.splits == 1;
+    g.slot = c;
+    return g.kb1 > g.kb0;
+  }
+  const long long it0 = sk_start(s, c), it1 = sk_start(s, c + 1);
+  long long it = it0;
+  for (int i = 0; i < q && it < it1; ++i) it = (it / s.kb_total + 1) * s.kb_total;
+  if (it >= it1) return false;
+  g.tile = static_cast<int>(it / s.kb_total);
+  g.kb0 = static_cast<int>(it % s.kb_total);
+  const long long end = min(it1, static_cast<long long>(g.tile + 1) * s.kb_total);
+  g.kb1 = static_cast<int>(end - static_cast<long long>(g.tile) * s.kb_total);
+  g.full = g.kb0 == 0 && g.kb1 == s.kb_total;
+  g.slot = 2 * c + (q == 0 ? 0 : 1);
+  return true;
+}
+
+// First CTA whose stream-K range reaches into the iterations starting at t0.
+__device__ __forceinline__ int sk_first_contributor(const Sched& s, long long t0) {
+  int lo = static_cast<int>(t0 * s.grid / s.iters);
+  while (lo > 0 && sk_start(s, lo) > t0) --lo;
+  while (lo + 1 < s.grid && sk_start(s, lo + 1) <= t0) ++lo;
+  return lo;
+}
 
 __device__ __forceinline__ uint64_t drain_ns(uint64_t wait_ns) {
   return wait_ns > 1000000000ull ? wait_ns : 1000000000ull;
@@ -73,12 +164,8 @@ __device__ __forceinline__ float gelu_erf(float v) {
   return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
 }
 
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
-  return *reinterpret_cast<__half2*>(&u);
-}
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
-  return *reinterpret_cast<uint32_t*>(&h);
-}
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
 // 8 codes (tiled nibble order) -> 8 fp16 values code * s + m.
 __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2, __half2 m2) {
@@ -91,6 +178,75 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2, __half2 m2) {
   return r;
 }
 
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
+
+__device__ __forceinline__ bool al16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+__device__ __forceinline__ void load_h16(const __half* src, int count, float (&v)[16]) {
+  if (count == 16 && al16(src)) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float2 f = __half22float2(u32_as_h2(w[u]));
+      v[2 * u] = f.x;
+      v[2 * u + 1] = f.y;
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = u < count ? __half2float(src[u]) : 0.f;
+  }
+}
+
+// Epilogue for 16 consecutive output features f0..f0+15 of one token: every
+// load is issued before any store, and full aligned rows use 16-byte vectors.
+__device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16], int tok, int f0) {
+  const int count = min(16, p.n - f0);
+  if (p.epi & EPI_F32_OUT) {
+    float* dst = p.yf + static_cast<size_t>(tok) * p.ldyf + f0;
+    if (count == 16 && al16(dst)) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        reinterpret_cast<float4*>(dst)[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+    } else {
+      for (int u = 0; u < count; ++u) dst[u] = v[u];
+    }
+    return;
+  }
+  float bv[16], rv[16];
+  if (p.epi & EPI_BIAS) {
+    load_h16(p.bias + f0, count, bv);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) bv[u] = 0.f;
+  }
+  if (p.epi & EPI_RESIDUAL) {
+    load_h16(p.residual + static_cast<size_t>(tok) * p.ld_res + f0, count, rv);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) rv[u] = 0.f;
+  }
+  uint32_t packed[8];
+#pragma unroll
+  for (int u = 0; u < 16; u += 2) {
+    float a = v[u] + bv[u], b = v[u + 1] + bv[u + 1];
+    if (p.epi & EPI_GELU) {
+      a = gelu_erf(a);
+      b = gelu_erf(b);
+    }
+    packed[u / 2] = h2_as_u32(__floats2half2_rn(a + rv[u], b + rv[u + 1]));
+  }
+  __half* dst = p.y + static_cast<size_t>(tok) * p.ldy + f0;
+  if (count == 16 && al16(dst)) {
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+  } else {
+    const __half* hv = reinterpret_cast<const __half*>(packed);
+    for (int u = 0; u < count; ++u) dst[u] = hv[u];
+  }
+}
+
 template <bool kW4>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
@@ -98,199 +254,318 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int S = p.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * p.stage_bytes);
-  uint64_t* afull = full + S;
-  uint64_t* empty = afull + S;
-  uint64_t* accum = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum + 1);
+  const int SL = p.load_stages, SA = p.a_stages;
+  uint8_t* a_ring = smem;                     // SA x 16 KB (4-bit weights only)
+  uint8_t* l_ring = smem + SA * kATileBytes;  // SL x load_stage_bytes
+  uint64_t* full = reinterpret_cast<uint64_t*>(l_ring + SL * p.load_stage_bytes);
+  uint64_t* empty = full + SL;
+  uint64_t* afull = empty + SL;
+  uint64_t* aempty = afull + SA;
+  uint64_t* accf = aempty + SA;  // [2]
+  uint64_t* acce = accf + 2;     // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
+  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + kBarrierBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_tile = blockIdx.x;
-  const int t_tile = blockIdx.y;
-  const int kb0 = blockIdx.z * p.kb_per_split;
-  const int kb1 = min(p.kb_total, kb0 + p.kb_per_split);
-  const int nkb = kb1 - kb0;
+  const int cta = blockIdx.x;
   const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;
+  // load stage layout: 4-bit = [B tile | raw chunk]; fp16 = [A tile | B tile]
+  const uint32_t b_off = kW4 ? 0u : static_cast<uint32_t>(kATileBytes);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
+    for (int s = 0; s < SL; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&afull[s], kConsumers);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accum, 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&afull[s], kDequantThreads);
+      mbar_init(&aempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accf[b], 1);
+      mbar_init(&acce[b], kEpiThreads);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_alloc(tmem_slot, 2 * p.tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_d = *tmem_slot;
+  const uint32_t tmem_base = *tmem_slot;
+  const Sched& sc = p.sc;
 
   if (warp == 0) {
+    // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmap_x);
       if (!kW4) prefetch_tmap(&tmap_w);
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % S;
-        const uint32_t r = static_cast<uint32_t>(i / S);
-        if (!mbar_wait(&empty[s], (r & 1u) ^ 1u, p.wait_ns)) {
-          set_error(p.err, DEV_TIMEOUT_PRODUCER);
-          *abort_flag = 1;
-          break;
+      int i = 0;
+      Ring rl;
+      Seg g;
+      bool stop = false;
+      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
+        const int n_tile = g.tile % sc.n_tiles;
+        const int t_tile = g.tile / sc.n_tiles;
+        for (int kb = g.kb0; kb < g.kb1; ++kb, ++i, rl.next(SL)) {
+          const int s = rl.s;
+          if (!mbar_wait(&empty[s], rl.ph ^ 1u, p.wait_ns)) {
+            set_error(p.err, DEV_TIMEOUT_PRODUCER);
+            *abort_flag = 1;
+          }
+          if (*abort_flag) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = l_ring + s * p.load_stage_bytes;
+          if (kW4) {
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kTileBytes) + b_bytes);
+            bulk_load(st + b_bytes, p.wq + (static_cast<size_t>(n_tile) * sc.kb_total + kb) * kTileBytes,
+                      kTileBytes, &full[s], pol_w);
+          } else {
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kATileBytes) + b_bytes);
+            tma_load_2d(st, &tmap_w, &full[s], kb * 64, n_tile * 128, pol_w);
+          }
+          tma_load_2d(st + b_off, &tmap_x, &full[s], kb * 64, t_tile * p.tok_tile, pol_x);
         }
-        if (*abort_flag) break;
-        uint8_t* st = smem + s * p.stage_bytes;
-        const int kb = kb0 + i;
-        if (kW4) {
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kTileBytes) + b_bytes);
-          bulk_load(st + kATileBytes + b_bytes,
-                    p.wq + (static_cast<size_t>(n_tile) * p.kb_total + kb) * kTileBytes, kTileBytes,
-                    &full[s], pol_w);
-        } else {
-          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kATileBytes) + b_bytes);
-          tma_load_2d(st, &tmap_w, &full[s], kb * 64, n_tile * 128, pol_w);
-        }
-        tma_load_2d(st + kATileBytes, &tmap_x, &full[s], kb * 64, t_tile * p.tok_tile, pol_x);
-        ++issued;
       }
-      // Never leave the CTA with bulk copies still landing in its shared memory
-      // (the drain keeps a deadline of its own so a short wait limit cannot cut
-      // it short).
-      for (int j = max(0, issued - S); j < issued; ++j)
-        mbar_wait(&full[j % S], static_cast<uint32_t>(j / S) & 1u, drain_ns(p.wait_ns));
+      // Never leave the CTA with bulk copies still landing in its shared memory.
+      for (int j = max(0, i - SL); j < i; ++j)
+        mbar_wait(&full[j % SL], static_cast<uint32_t>(j / SL) & 1u, drain_ns(p.wait_ns));
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % S;
-        const uint32_t r = static_cast<uint32_t>(i / S);
-        if (!mbar_wait(kW4 ? &afull[s] : &full[s], r & 1u, p.wait_ns)) {
+      Ring rl, ra;
+      Seg g;
+      bool stop = false;
+      for (int q = 0; get_seg(sc, cta, q, g); ++q) {
+        const int buf = q & 1;
+        if (!stop && !mbar_wait(&acce[buf], (static_cast<uint32_t>(q >> 1) & 1u) ^ 1u, p.wait_ns)) {
           set_error(p.err, DEV_TIMEOUT_MMA);
           *abort_flag = 1;
-          break;
         }
-        if (*abort_flag) break;
+        if (*abort_flag) stop = true;
         tc_fence_after();
-        uint8_t* st = smem + s * p.stage_bytes;
-        const uint64_t adesc = sw128_kmajor_desc(smem_u32(st));
-        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(st + kATileBytes));
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.tmem_cols;
+        for (int kb = g.kb0; kb < g.kb1 && !stop; ++kb, rl.next(SL), ra.next(SA)) {
+          const int s = rl.s;
+          const int sa = kW4 ? ra.s : 0;
+          const bool ok = kW4 ? mbar_wait(&afull[sa], ra.ph, p.wait_ns) : mbar_wait(&full[s], rl.ph, p.wait_ns);
+          if (!ok) {
+            set_error(p.err, DEV_TIMEOUT_MMA);
+            *abort_flag = 1;
+          }
+          if (*abort_flag) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          uint8_t* st = l_ring + s * p.load_stage_bytes;
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(kW4 ? a_ring + sa * kATileBytes : st));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(st + b_off));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f16_ss(tmem_d, adesc + 2 * kk, bdesc + 2 * kk, idesc, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&empty[s]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > g.kb0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+          if (kW4) mma_commit(&aempty[sa]);
+        }
+        // Every segment ends with a commit, also after an abort, so the
+        // epilogue and the teardown never wait on a barrier nobody signals.
+        mma_commit(&accf[buf]);
       }
-      mma_commit(accum);
     }
-  } else {
-    const int ct = threadIdx.x - 64;
+  } else if (warp < kEpiWarp0) {
+    // ------------------------------------------------------------ dequantize
     if (kW4) {
+      const int ct = threadIdx.x - 64;
       const int row = ct >> 1;
       const int hf = ct & 1;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % S;
-        const uint32_t r = static_cast<uint32_t>(i / S);
-        if (!mbar_wait(&full[s], r & 1u, p.wait_ns)) {
-          set_error(p.err, DEV_TIMEOUT_CONSUMER);
-          *abort_flag = 1;
-          break;
-        }
-        if (*abort_flag) break;
-        uint8_t* st = smem + s * p.stage_bytes;
-        const uint8_t* raw = st + kATileBytes + b_bytes;
-        const uint4 c = *reinterpret_cast<const uint4*>(raw + row * 32 + hf * 16);
-        const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
-        const __half2 m2 = __low2half2(mm);
-        const __half2 s2 = __high2half2(mm);
-        uint8_t* arow = st + row * 128;
-        const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+      Ring rl, ra;
+      Seg g;
+      bool stop = false;
+      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
+        for (int kb = g.kb0; kb < g.kb1; ++kb, rl.next(SL), ra.next(SA)) {
+          const int s = rl.s;
+          const int sa = ra.s;
+          bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
+          ok = ok && mbar_wait(&aempty[sa], ra.ph ^ 1u, p.wait_ns);
+          if (!ok) {
+            set_error(p.err, DEV_TIMEOUT_CONSUMER);
+            *abort_flag = 1;
+          }
+          if (*abort_flag) {
+            stop = true;
+            break;
+          }
+          const uint8_t* raw = l_ring + s * p.load_stage_bytes + b_bytes;
+          const uint4 c = *reinterpret_cast<const uint4*>(raw + row * 32 + hf * 16);
+          const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
+          const __half2 m2 = __low2half2(mm);
+          const __half2 s2 = __high2half2(mm);
+          uint8_t* arow = a_ring + sa * kATileBytes + row * 128;
+          const uint32_t words[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int phys = (hf * 4 + j) ^ (row & 7);
-          *reinterpret_cast<uint4*>(arow + phys * 16) = dequant8(words[j], s2, m2);
+          for (int j = 0; j < 4; ++j) {
+            const int phys = (hf * 4 + j) ^ (row & 7);
+            *reinterpret_cast<uint4*>(arow + phys * 16) = dequant8(words[j], s2, m2);
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&afull[sa]);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&afull[s]);
       }
     }
-    // epilogue
-    const bool ok = mbar_wait(accum, 0, p.wait_ns);
-    if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
-    tc_fence_after();
-    if (ok && !*abort_flag) {
-      const int q = warp & 3;
-      const int wg = (warp - 2) >> 2;
-      const int feat = n_tile * 128 + q * 32 + lane;
-      const bool fvalid = feat < p.n;
-      const uint32_t tbase = tmem_d + (static_cast<uint32_t>(q * 32) << 16);
-      float bias_v = 0.f;
-      if ((p.epi & EPI_BIAS) && fvalid && !p.splitk) bias_v = __half2float(p.bias[feat]);
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - kEpiWarp0 * 32;
+    const int qd = warp & 3;  // TMEM lane quarter this warp may access
+    Seg g;
+    for (int q = 0; get_seg(sc, cta, q, g); ++q) {
+      const int buf = q & 1;
+      const bool ok = mbar_wait(&accf[buf], static_cast<uint32_t>(q >> 1) & 1u, drain_ns(p.wait_ns));
+      if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
+      tc_fence_after();
+      const bool aborted = !ok || *abort_flag;
+      const int n_tile = g.tile % sc.n_tiles;
+      const int t_tile = g.tile / sc.n_tiles;
+      const int frow = qd * 32 + lane;  // feature row inside the tile
+      float* stg = epi_stage + (warp - kEpiWarp0) * 16 * 33;
       const int tok0 = t_tile * p.tok_tile;
-      for (int c0 = wg * 16; c0 < p.tok_tile; c0 += 32) {
+      const uint32_t tbase = tmem_base + static_cast<uint32_t>(buf) * p.tmem_cols +
+                             (static_cast<uint32_t>(qd * 32) << 16);
+      float* slot = g.full ? nullptr : p.partials + static_cast<size_t>(g.slot) * p.tok_tile * 128;
+      for (int c0 = 0; c0 < p.tok_tile && !aborted; c0 += 16) {
         uint32_t rr[16];
         tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
         tmem_ld_wait();
-        if (!fvalid) continue;
+        if (slot) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int tok = tok0 + c0 + j;
-          if (tok >= p.m) break;
-          float v = __uint_as_float(rr[j]);
-          if (p.splitk) {
-            atomicAdd(p.yf + static_cast<size_t>(tok) * p.ldyf + feat, v);
-          } else if (p.epi & EPI_F32_OUT) {
-            p.yf[static_cast<size_t>(tok) * p.ldyf + feat] = v;
-          } else {
-            v += bias_v;
-            if (p.epi & EPI_GELU) v = gelu_erf(v);
-            if (p.epi & EPI_RESIDUAL)
-              v += __half2float(p.residual[static_cast<size_t>(tok) * p.ld_res + feat]);
-            p.y[static_cast<size_t>(tok) * p.ldy + feat] = __float2half_rn(v);
+          for (int j = 0; j < 16; ++j) slot[(c0 + j) * 128 + frow] = __uint_as_float(rr[j]);
+        } else {
+          // transpose 32 features x 16 tokens through shared memory so each
+          // lane finishes 16 consecutive features of one token
+#pragma unroll
+          for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = __uint_as_float(rr[j]);
+          __syncwarp();
+          const int jt = lane >> 1, hf = lane & 1;
+          const int tok = tok0 + c0 + jt;
+          const int f0 = n_tile * 128 + qd * 32 + hf * 16;
+          if (tok < p.m && f0 < p.n) {
+            float v[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) v[u] = stg[jt * 33 + hf * 16 + u];
+            store_row16(p, v, tok, f0);
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acce[buf]);
+      if (slot == nullptr || aborted) continue;
+      // Partial tile: publish it, count it, and let the last contributor finish.
+      __threadfence();
+      epi_bar();
+      if (et == 0) {
+        int ncontrib;
+        if (sc.mode == SCHED_SPLITS) {
+          ncontrib = sc.splits;
+        } else {
+          const long long t0 = static_cast<long long>(g.tile) * sc.kb_total;
+          const int lo = sk_first_contributor(sc, t0);
+          int hi = lo;
+          while (hi + 1 < sc.grid && sk_start(sc, hi + 1) < t0 + sc.kb_total) ++hi;
+          ncontrib = hi - lo + 1;
+        }
+        const int old = atomicAdd(&p.counters[g.tile], 1);
+        *last_flag = old == ncontrib - 1;
+      }
+      epi_bar();
+      const bool last = *last_flag;
+      epi_bar();  // everyone has read the flag before it can be rewritten
+      if (!last) continue;
+      __threadfence();
+      int slots[kMaxContrib];
+      int ns = 0;
+      if (sc.mode == SCHED_SPLITS) {
+        for (int part = 0; part < sc.splits && ns < kMaxContrib; ++part) slots[ns++] = g.tile * sc.splits + part;
+      } else {
+        const long long t0 = static_cast<long long>(g.tile) * sc.kb_total;
+        for (int c = sk_first_contributor(sc, t0); c < sc.grid && sk_start(sc, c) < t0 + sc.kb_total &&
+                                                   ns < kMaxContrib;
+             ++c)
+          slots[ns++] = 2 * c + (sk_start(sc, c) >= t0 ? 0 : 1);
+      }
+      // Sum the slots in contributor order with coalesced 16-byte loads (two
+      // contributors in flight): thread et finishes features 16*(et%8)..+15 of
+      // tokens et/8, et/8 + 16, ... of the tile.
+      const int fg = (et & 7) * 16;
+      const int tsub = et >> 3;
+      const int f0 = n_tile * 128 + fg;
+      for (int c = tsub; c < p.tok_tile; c += 16) {
+        float acc[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+        int k = 0;
+        for (; k + 1 < ns; k += 2) {
+          const float4* b0 = reinterpret_cast<const float4*>(
+              p.partials + (static_cast<size_t>(slots[k]) * p.tok_tile + c) * 128 + fg);
+          const float4* b1 = reinterpret_cast<const float4*>(
+              p.partials + (static_cast<size_t>(slots[k + 1]) * p.tok_tile + c) * 128 + fg);
+          float4 v0[4], v1[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            v0[u] = __ldcg(b0 + u);
+            v1[u] = __ldcg(b1 + u);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            acc[4 * u] += v0[u].x + v1[u].x;
+            acc[4 * u + 1] += v0[u].y + v1[u].y;
+            acc[4 * u + 2] += v0[u].z + v1[u].z;
+            acc[4 * u + 3] += v0[u].w + v1[u].w;
           }
         }
+        if (k < ns) {
+          const float4* b0 = reinterpret_cast<const float4*>(
+              p.partials + (static_cast<size_t>(slots[k]) * p.tok_tile + c) * 128 + fg);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float4 v = __ldcg(b0 + u);
+            acc[4 * u] += v.x;
+            acc[4 * u + 1] += v.y;
+            acc[4 * u + 2] += v.z;
+            acc[4 * u + 3] += v.w;
+          }
+        }
+        const int tok = tok0 + c;
+        if (tok < p.m && f0 < p.n) store_row16(p, acc, tok, f0);
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
-    // The accumulator barrier completes only when every issued MMA has
-    // finished, so TMEM is never released under a running MMA.
-    if (lane == 0) mbar_wait(accum, 0, drain_ns(p.wait_ns));
+    // The last segment's accumulator commit completes only after every MMA of
+    // this CTA; wait for it so TMEM is never released under a running MMA.
+    if (lane == 0) {
+      Seg g;
+      int nq = 0;
+      while (get_seg(sc, cta, nq, g)) ++nq;
+      if (nq > 0) mbar_wait(&accf[(nq - 1) & 1], static_cast<uint32_t>((nq - 1) >> 1) & 1u, drain_ns(p.wait_ns));
+    }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_d, p.tmem_cols);
+    tmem_dealloc(tmem_base, 2 * p.tmem_cols);
   }
-}
-
-// Split-K finish: Y = epilogue(sum of partials).
-__global__ void splitk_finish_kernel(const float* __restrict__ acc, int m, int n, const __half* bias,
-                                     const __half* residual, int ld_res, __half* y, int ldy,
-                                     float* yf, int ldyf, int epi) {
-  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<size_t>(m) * n) return;
-  const int tok = static_cast<int>(idx / n);
-  const int feat = static_cast<int>(idx % n);
-  float v = acc[idx];
-  if (epi & EPI_F32_OUT) {
-    yf[static_cast<size_t>(tok) * ldyf + feat] = v;
-    return;
-  }
-  if (epi & EPI_BIAS) v += __half2float(bias[feat]);
-  if (epi & EPI_GELU) v = gelu_erf(v);
-  if (epi & EPI_RESIDUAL) v += __half2float(residual[static_cast<size_t>(tok) * ld_res + feat]);
-  y[static_cast<size_t>(tok) * ldy + feat] = __float2half_rn(v);
 }
 
 // ---------------------------------------------------------------------------
@@ -329,12 +604,16 @@ bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, i
 }
 
 struct Plan {
-  int tok_tile, tok_tiles, n_tiles, splits, kb_per_split, stages;
-  uint32_t stage_bytes;
+  int tok_tile, tok_tiles, n_tiles;
+  Sched sc;
+  int load_stages, a_stages;
+  uint32_t load_stage_bytes;
   size_t smem;
+  size_t partial_bytes, counter_bytes;
 };
 
 int round_up(int a, int b) { return (a + b - 1) / b * b; }
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_tile) {
   Plan P{};
@@ -351,19 +630,51 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   }
   P.n_tiles = (n + 127) / 128;
   const int tiles = P.n_tiles * P.tok_tiles;
-  int splits = 1;
-  if (force_splits > 0) {
-    splits = force_splits;
+  const int sms = runtime().num_sms;
+  Sched& s = P.sc;
+  s.tiles = tiles;
+  s.n_tiles = P.n_tiles;
+  s.kb_total = kb_total;
+  s.iters = static_cast<long long>(tiles) * kb_total;
+  s.splits = 1;
+  s.per = kb_total;
+  const size_t tile_bytes = static_cast<size_t>(P.tok_tile) * 128 * sizeof(float);
+  if (force_splits > 1) {
+    s.mode = SCHED_SPLITS;
+    s.per = (kb_total + force_splits - 1) / force_splits;
+    s.splits = min(kMaxContrib, (kb_total + s.per - 1) / s.per);
+    s.per = (kb_total + s.splits - 1) / s.splits;
+    s.grid = tiles * s.splits;
+    if (s.splits > 1) P.partial_bytes = static_cast<size_t>(s.grid) * tile_bytes;
+    else s.mode = SCHED_TILES, s.grid = min(tiles, sms);
+  } else if (force_splits == 1 || tiles >= 16 * sms ||
+             tiles % std::max<long long>(1, std::min<long long>(sms, s.iters / kMinItersPerCta)) == 0) {
+    // many tiles, or whole tiles already divide evenly over the CTAs stream-K would use
+    s.mode = SCHED_TILES;
+    s.grid = min(tiles, sms);
   } else {
-    const int sms = runtime().num_sms;
-    if (tiles < sms) splits = min(max(1, kb_total / 8), (sms + tiles - 1) / tiles);
+    s.mode = SCHED_STREAMK;
+    s.grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, s.iters / kMinItersPerCta)));
+    // A tile is shared by at most ceil(kb_total / (iters / grid)) + 1 CTAs.
+    const long long per_cta = s.iters / s.grid;
+    if ((kb_total + per_cta - 1) / per_cta + 1 > kMaxContrib)
+      s.grid = static_cast<int>(std::max<long long>(1, s.iters * (kMaxContrib - 2) / kb_total));
+    P.partial_bytes = static_cast<size_t>(2) * s.grid * tile_bytes;
   }
-  splits = max(1, min(splits, kb_total));
-  P.kb_per_split = (kb_total + splits - 1) / splits;
-  P.splits = (kb_total + P.kb_per_split - 1) / P.kb_per_split;
-  P.stage_bytes = static_cast<uint32_t>(kATileBytes + P.tok_tile * 128 + (w_bits == 4 ? kRawBytes : 0));
-  P.stages = min(8, static_cast<int>((kMaxSmem - 1024 - kBarrierBytes) / P.stage_bytes));
-  P.smem = static_cast<size_t>(P.stages) * P.stage_bytes + 1024 + kBarrierBytes;
+  if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * sizeof(int);
+  const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
+  if (w_bits == 4) {
+    P.a_stages = P.tok_tile > 128 && P.tok_tile != 144 ? 2 : 3;
+    P.load_stage_bytes = static_cast<uint32_t>(P.tok_tile * 128 + kRawBytes);
+    P.load_stages = min(kMaxLoadStages, static_cast<int>((budget - P.a_stages * kATileBytes) / P.load_stage_bytes));
+  } else {
+    P.a_stages = 0;
+    P.load_stage_bytes = static_cast<uint32_t>(kATileBytes + P.tok_tile * 128);
+    P.load_stages = min(kMaxLoadStages, static_cast<int>(budget / P.load_stage_bytes));
+  }
+  P.load_stages = min(P.load_stages, static_cast<int>((budget - P.a_stages * kATileBytes) / P.load_stage_bytes));
+  P.smem = static_cast<size_t>(P.a_stages) * kATileBytes + static_cast<size_t>(P.load_stages) * P.load_stage_bytes +
+           1024 + kBarrierBytes + kEpiStageBytes;
   return P;
 }
 
@@ -381,13 +692,15 @@ cudaError_t configure_once() {
 
 size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits) {
   const Plan P = make_plan(m, n, k, w_bits, force_splits, 0);
-  return P.splits > 1 ? static_cast<size_t>(m) * n * sizeof(float) : 0;
+  if (P.partial_bytes == 0) return 0;
+  return align256(P.partial_bytes) + align256(P.counter_bytes);
 }
 
 cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaStream_t s) {
   if (a.m == 0 || a.n == 0) return cudaSuccess;
   const Plan P = make_plan(a.m, a.n, a.k, a.w_bits, a.force_splits, a.force_tok_tile);
   const bool w4 = a.w_bits == 4;
+  if (P.load_stages < 2) return cudaErrorInvalidValue;
   cudaError_t e = w4 ? configure_once<true>() : configure_once<false>();
   if (e != cudaSuccess) return e;
   CUtensorMap tx, tw;
@@ -402,47 +715,39 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.m = a.m;
   p.n = a.n;
   p.k = a.k;
-  p.kb_total = a.k / 64;
-  p.kb_per_split = P.kb_per_split;
   p.tok_tile = P.tok_tile;
-  p.stages = P.stages;
-  p.stage_bytes = P.stage_bytes;
+  p.load_stages = P.load_stages;
+  p.a_stages = P.a_stages;
+  p.load_stage_bytes = P.load_stage_bytes;
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
   p.tmem_cols = cols;
+  p.sc = P.sc;
   p.bias = a.bias;
   p.residual = a.residual;
   p.ld_res = a.ld_res;
   p.epi = a.epi;
   p.wait_ns = runtime().wait_limit_ns;
   p.err = runtime().err;
-  const bool split = P.splits > 1;
-  if (split) {
-    const size_t need = static_cast<size_t>(a.m) * a.n * sizeof(float);
-    if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
-    e = cudaMemsetAsync(ws, 0, need, s);
-    if (e != cudaSuccess) return e;
-    p.splitk = 1;
-    p.yf = static_cast<float*>(ws);
-    p.ldyf = a.n;
-  } else if (a.epi & EPI_F32_OUT) {
+  if (a.epi & EPI_F32_OUT) {
     p.yf = static_cast<float*>(a.y);
     p.ldyf = a.ldy;
   } else {
     p.y = static_cast<__half*>(a.y);
     p.ldy = a.ldy;
   }
-  dim3 grid(P.n_tiles, P.tok_tiles, P.splits);
+  if (P.partial_bytes > 0) {
+    const size_t need = align256(P.partial_bytes) + align256(P.counter_bytes);
+    if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
+    p.partials = static_cast<float*>(ws);
+    p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + align256(P.partial_bytes));
+    e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
+    if (e != cudaSuccess) return e;
+  }
   if (w4)
-    gemm_tc_kernel<true><<<grid, kThreads, P.smem, s>>>(tx, tw, p);
+    gemm_tc_kernel<true><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
   else
-    gemm_tc_kernel<false><<<grid, kThreads, P.smem, s>>>(tx, tw, p);
-  e = launched();
-  if (e != cudaSuccess || !split) return e;
-  const size_t total = static_cast<size_t>(a.m) * a.n;
-  splitk_finish_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(
-      static_cast<const float*>(ws), a.m, a.n, a.bias, a.residual, a.ld_res, static_cast<__half*>(a.y),
-      a.ldy, static_cast<float*>(a.y), a.ldy, a.epi);
+    gemm_tc_kernel<false><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
   return launched();
 }
 

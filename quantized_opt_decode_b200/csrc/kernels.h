@@ -47,6 +47,10 @@ cudaError_t launch_pack_weight(const uint8_t* codes, const __half* mn, const __h
 cudaError_t launch_quantize_weight(const __half* w, int n_out, int k_in, uint8_t* packed,
                                    cudaStream_t s);
 
+// Slots per (sequence, head) of the token-interleaved 4-bit V codes: max_len
+// rounded up to whole blocks of 8 tokens.
+__host__ __device__ inline int kv_pad_len(int max_len) { return (max_len + 7) & ~7; }
+
 // KV cache append (quantize on append in 4-bit mode)
 struct KvView {
   void* k;        // 4-bit: codes [b][a][L][d/2]; 16-bit: fp16 [b][a][L][d]

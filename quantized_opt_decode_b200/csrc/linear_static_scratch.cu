@@ -11,8 +11,8 @@
 // partial sums in a fixed array compiled into the library instead.
 //
 // Properties a user must know:
-// * The array holds kStaticScratchBytes (8 MiB), i.e. m * n <= 2,097,152 fp32
-//   partial sums whenever K is split; larger requests are rejected with
+// * The array holds kStaticScratchBytes (8 MiB) of fp32 partial tiles; a shape
+//   whose K-split scratch (flexq_linear_workspace) is larger is rejected with
 //   FLEXQ_ERR_INVALID before anything is launched.  Every GPU that loads the
 //   library keeps these 8 MiB reserved until the process exits.
 // * The first call on a device looks up the array's device address (once per
@@ -81,8 +81,8 @@ extern "C" flexq_status flexq_linear_static_scratch(const void* x_dev, int ldx, 
   if (need > kStaticScratchBytes) {
     char msg[200];
     snprintf(msg, sizeof(msg),
-             "K-split partial sums need %zu bytes; the static scratch holds %zu (m*n <= %zu when K is split)",
-             need, kStaticScratchBytes, kStaticScratchBytes / sizeof(float));
+             "K-split partial sums need %zu bytes; the static scratch holds %zu", need,
+             kStaticScratchBytes);
     set_last_error(msg);
     return FLEXQ_ERR_INVALID;
   }

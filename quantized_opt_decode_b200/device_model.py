@@ -37,7 +37,9 @@ class KVCache:
         slots = b * cfg.heads * max_len
         if cfg.kv_bits == 4:
             self.k = torch.zeros(slots * d // 2, dtype=torch.uint8, device=device)
-            self.v = torch.zeros_like(self.k)
+            # V codes: whole 8-token blocks of 32-bit words (token-interleaved)
+            l8 = (max_len + 7) // 8 * 8
+            self.v = torch.zeros(b * cfg.heads * l8 * d // 2, dtype=torch.uint8, device=device)
             self.k_meta = torch.zeros(slots * (d // 64) * 2, dtype=torch.float16, device=device)
             self.v_meta = torch.zeros_like(self.k_meta)
         else:
@@ -51,9 +53,9 @@ class KVCache:
                                   b, max_len)
 
     def nbytes(self) -> int:
-        n = self.k.numel() * self.k.element_size() * 2
+        n = self.k.numel() * self.k.element_size() + self.v.numel() * self.v.element_size()
         if self.k_meta is not None:
-            n += self.k_meta.numel() * 2 * 2
+            n += (self.k_meta.numel() + self.v_meta.numel()) * 2
         return n
 
 

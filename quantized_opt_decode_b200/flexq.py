@@ -80,7 +80,7 @@ _SIGS = {
     "flexq_packed_weight_bytes": ([C.c_int, C.c_int], C.c_size_t),
     "flexq_pack_weight_q4": ([VP, VP, VP, C.c_int, C.c_int, VP, VP], C.c_int),
     "flexq_quantize_weight_q4": ([VP, C.c_int, C.c_int, VP, VP], C.c_int),
-    "flexq_linear_workspace": ([C.c_int, C.c_int, C.c_int, C.c_int], C.c_size_t),
+    "flexq_linear_workspace": ([C.c_int, C.c_int, C.c_int, C.c_int, C.c_int], C.c_size_t),
     "flexq_linear": ([VP, C.c_int, VP, C.c_int, C.c_int, C.c_int, C.c_int, VP, VP, C.c_int,
                       C.c_int, VP, C.c_int, VP, C.c_size_t, C.c_int, VP], C.c_int),
     "flexq_linear_static_scratch": ([VP, C.c_int, VP, C.c_int, C.c_int, C.c_int, C.c_int, VP, VP,
@@ -185,8 +185,8 @@ def flexq_quantize_weight_q4(w, n_out, k_in, packed, stream=None):
     _check(_lib.flexq_quantize_weight_q4(_p(w), n_out, k_in, _p(packed), _s(stream)))
 
 
-def flexq_linear_workspace(m, n, k, w_bits) -> int:
-    return _lib.flexq_linear_workspace(m, n, k, w_bits)
+def flexq_linear_workspace(m, n, k, w_bits, force_splits=0) -> int:
+    return _lib.flexq_linear_workspace(m, n, k, w_bits, force_splits)
 
 
 def flexq_linear(x, ldx, w, w_bits, m, n, k, bias, residual, ld_res, epilogue, y, ldy,

@@ -78,7 +78,7 @@ def bench_gemm(p, kind, M, reps, warmup, stream, splits):
     bias = torch.zeros(n, dtype=torch.float16, device="cuda")
     res = torch.zeros(M, n, dtype=torch.float16, device="cuda")
     y = torch.empty(M, n, dtype=torch.float16, device="cuda")
-    ws_n = max(M * n * 4, 1)
+    ws_n = max(fq.flexq_linear_workspace(M, n, k, p["w_bits"], splits), 1)
     ws = workspace(ws_n)
     epi = fq.EPI_BIAS | GEMMS[kind][2]
 
@@ -170,7 +170,7 @@ def bench_lm_head(p, b, reps, warmup, stream):
     x = torch.empty(b, h, dtype=torch.float16, device="cuda")
     fq.flexq_synth_normal_f16(x, b * h, synth.config_seed(p), 992, 0, 1.0, 0.0, stream)
     y = torch.empty(b, V, dtype=torch.float32, device="cuda")
-    ws_n = max(fq.flexq_linear_workspace(b, V, h, 16), 1)
+    ws_n = max(fq.flexq_linear_workspace(b, V, h, 16, 0), 1)
     ws = workspace(ws_n)
 
     def run():

@@ -64,3 +64,16 @@ def tiled_to_canonical(packed: np.ndarray, n_out: int, k_in: int):
     can = (q[:, 0::2] | (q[:, 1::2] << 4)).astype(np.uint8)
     meta = meta.transpose(0, 2, 1, 3).reshape(nt * 128, kb, 2)[:n_out]
     return can, meta[..., 0].copy(), meta[..., 1].copy()
+
+
+def v_words_to_canonical(words: np.ndarray, b: int, heads: int, max_len: int, d: int):
+    """Reads the token-interleaved 4-bit V layout (include/flexq.h: nibble k of
+    word (block, e) = token 8*block + k at dimension e) back into canonical
+    per-token rows [b][heads][max_len][d/2] (low nibble = even element)."""
+    l8 = (max_len + 7) // 8 * 8
+    w = np.ascontiguousarray(words).view(np.uint32).reshape(b, heads, l8 // 8, d)
+    codes = np.zeros((b, heads, l8 // 8, 8, d), np.uint8)
+    for k in range(8):
+        codes[:, :, :, k, :] = (w >> np.uint32(4 * k)) & np.uint32(0xF)
+    codes = codes.reshape(b, heads, l8, d)[:, :, :max_len]
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)

@@ -47,7 +47,7 @@ def _linear_case(m, n, k, w_bits, epi, splits, seed):
         w_eff = w.astype(np.float64)
     f32 = epi == fq.EPI_F32_OUT
     y = torch.empty(m, n, dtype=torch.float32 if f32 else torch.float16, device="cuda")
-    ws_bytes = max(m * n * 4, 1)
+    ws_bytes = max(fq.flexq_linear_workspace(m, n, k, w_bits, splits), 1)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     fq.flexq_linear(to_dev(x), k, wd, w_bits, m, n, k, to_dev(bias), to_dev(res), n, epi, y, n,
                     ws, ws_bytes, splits)
@@ -105,12 +105,15 @@ def _dev_cache(cfg, b, max_len):
     return KVCache(cfg, b, max_len)
 
 
-@pytest.mark.parametrize("h,heads", [(256, 4), (512, 4)])
-def test_kv_append_bit_exact(h, heads):
-    """Each (sequence, head, token) row quantized exactly as the oracle does."""
+@pytest.mark.parametrize("h,heads,pos0,ntok", [(256, 4, 4, 5), (512, 4, 4, 5), (512, 4, 3, 21),
+                                                (256, 4, 0, 16), (512, 4, 7, 1), (512, 4, 8, 1)])
+def test_kv_append_bit_exact(h, heads, pos0, ntok):
+    """Each (sequence, head, token) row quantized exactly as the oracle does;
+    covers whole 8-token V blocks, ragged block edges and single tokens."""
+    from gpu_helpers import v_words_to_canonical
     cfg = _cfg(h, heads, 4)
-    b, ntok, L, pos0 = 3, 5, 12, 4
-    rng = np.random.default_rng(h)
+    b, L = 3, pos0 + ntok + 3
+    rng = np.random.default_rng(h + pos0 * 7 + ntok)
     ld = 3 * h
     rows = rng.standard_normal((b * ntok, ld)).astype(np.float16)
     dev = _dev_cache(cfg, b, L)
@@ -121,13 +124,19 @@ def test_kv_append_bit_exact(h, heads):
     oc.write("k", rows[:, h:2 * h].reshape(b, ntok, h), pos0)
     oc.write("v", rows[:, 2 * h:].reshape(b, ntok, h), pos0)
     d = h // heads
+    sl = slice(pos0, pos0 + ntok)
     kc = to_host(dev.k).reshape(b, heads, L, d // 2)
     km = to_host(dev.k_meta).reshape(b, heads, L, d // 64, 2)
-    vc = to_host(dev.v).reshape(b, heads, L, d // 2)
-    assert np.array_equal(kc, oc.t["k_codes"])
-    assert np.array_equal(vc, oc.t["v_codes"])
-    assert np.array_equal(km[..., 0].view(np.uint16), oc.t["k_min"].view(np.uint16))
-    assert np.array_equal(km[..., 1].view(np.uint16), oc.t["k_scale"].view(np.uint16))
+    vm = to_host(dev.v_meta).reshape(b, heads, L, d // 64, 2)
+    vc = v_words_to_canonical(to_host(dev.v), b, heads, L, d)
+    assert np.array_equal(kc[:, :, sl], oc.t["k_codes"][:, :, sl])
+    assert np.array_equal(vc[:, :, sl], oc.t["v_codes"][:, :, sl])
+    assert np.array_equal(km[:, :, sl, :, 0].view(np.uint16), oc.t["k_min"][:, :, sl].view(np.uint16))
+    assert np.array_equal(km[:, :, sl, :, 1].view(np.uint16), oc.t["k_scale"][:, :, sl].view(np.uint16))
+    assert np.array_equal(vm[:, :, sl, :, 0].view(np.uint16), oc.t["v_min"][:, :, sl].view(np.uint16))
+    assert np.array_equal(vm[:, :, sl, :, 1].view(np.uint16), oc.t["v_scale"][:, :, sl].view(np.uint16))
+    # slots outside the written range keep their (zero) codes
+    assert not vc[:, :, :pos0].any() and not vc[:, :, pos0 + ntok:].any()
 
 
 @pytest.mark.parametrize("h,heads,kv_bits,length", [(256, 4, 4, 1), (256, 4, 4, 37), (512, 4, 4, 545),

@@ -31,8 +31,7 @@ def _inputs(m, n, k, seed):
 def test_static_scratch_matches_workspace_linear_twice(m, n, k, splits):
     x, wq, bias, res = _inputs(m, n, k, m + n)
     epi = fq.EPI_BIAS | fq.EPI_RESIDUAL
-    need = fq.flexq_linear_workspace(m, n, k, 4)
-    ws_bytes = max(need, m * n * 4)
+    ws_bytes = max(fq.flexq_linear_workspace(m, n, k, 4, splits), 1)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
     ref = torch.empty(m, n, dtype=torch.float16, device="cuda")
     fq.flexq_linear(x, k, wq, 4, m, n, k, bias, res, n, epi, ref, n, ws, ws_bytes, splits)
