@@ -12,10 +12,11 @@
 // One output tile = 128 features x up to 256 tokens; the weight is the MMA's A
 // operand, so a small decode batch becomes the MMA's N.  A persistent CTA per
 // SM walks a list of (tile, k-block range) segments:
-//   warp 0      TMA producer: per 64-wide k-block one cp.async.bulk of the
-//               packed 4-bit chunk (codes + min/scale, 4608 contiguous bytes)
-//               or a tiled fp16 weight box, plus one 128-byte-swizzled
-//               cp.async.bulk.tensor of the activations, into a deep ring;
+//   warp 0      TMA producer: per k-step (one or two 64-wide k-blocks) one
+//               cp.async.bulk of the packed 4-bit chunks (codes + min/scale,
+//               4608 contiguous bytes per k-block) or tiled fp16 weight
+//               boxes, plus 128-byte-swizzled cp.async.bulk.tensor boxes of
+//               the activations, into a deep ring;
 //   warps 2-9   dequantize the chunk into a short ring of fp16 A tiles in the
 //               UMMA K-major SW128 layout ((code | 0x6400) is the fp16 value
 //               1024 + code; one half2 subtract and one half2 fused
@@ -23,11 +24,14 @@
 //   warp 1      owns TMEM (two accumulator buffers) and, from one thread,
 //               issues tcgen05.mma.kind::f16 (M=128, N=tokens, K=16) x 4 per
 //               k-block, releasing ring slots with tcgen05.commit;
+// Each mbarrier hand-off costs a few hundred cycles of latency in these
+// scalar role loops, so decode-sized tiles on 4-bit weights move two k-blocks
+// per stage (half the hand-offs per tile).
 //   warps 10-13 epilogue: tcgen05.ld, + bias, GELU, + residual, fp16 or fp32
 //               store; overlaps the next segment's main loop.
 // Scheduling: whole tiles round-robin over the SMs when there are many; when
 // the grid is small (decode), each SM takes an equal share of all k-blocks
-// (stream-K), so tiles may be split across CTAs.  A partial tile is written
+// (stream-K, in units of k-steps), so tiles may be split across CTAs.  A partial tile is written
 // to a per-contributor fp32 slot; the contributor that arrives last (an atomic
 // counter per tile) sums the slots in contributor order and applies the
 // epilogue, so results do not depend on timing.
@@ -48,9 +52,8 @@ constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
 constexpr int kATileBytes = 128 * 64 * 2;
-constexpr int kRawBytes = 5120;  // kTileBytes rounded up to keep 1 KB alignment
 constexpr int kMaxSmem = 227 * 1024;
-constexpr int kBarrierBytes = 512;
+constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
 constexpr int kEpiStageBytes = 4 * 16 * 33 * 4;  // per epilogue warp: 16 tokens x 33 floats
 constexpr int kMaxLoadStages = 16;
 constexpr int kMinItersPerCta = 8;
@@ -72,9 +75,15 @@ struct GemmParams {
   const uint8_t* wq;
   int m, n, k;
   int tok_tile;
+  int kb_real;  // 64-wide k-blocks of K
   int load_stages, a_stages;
   uint32_t load_stage_bytes;
-  uint32_t tmem_cols;  // per accumulator buffer
+  int n_sub;               // 128-row weight sub-tiles (ceil(n / 128))
+  uint32_t acc_cols;       // TMEM columns of one accumulator set (all M sub-tiles)
+  uint32_t m_stride;       // TMEM column offset between M sub-tiles
+  uint32_t tmem_alloc;     // columns allocated (power of two)
+  int nbuf;                // accumulator sets (2 = epilogue overlaps the next segment)
+  uint32_t a_col0;         // first TMEM column of the A ring (tensor-memory A)
   Sched sc;
   const __half* bias;
   const __half* residual;
@@ -180,6 +189,21 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2, __half2 m2) {
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
+// Barrier over the epilogue threads that also ORs a predicate across them, so
+// a branch taken on it is uniform (no thread skips a later epi_bar).
+__device__ __forceinline__ bool epi_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ bool al16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
 
 __device__ __forceinline__ void load_h16(const __half* src, int count, float (&v)[16]) {
@@ -247,16 +271,32 @@ __device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16],
   }
 }
 
-template <bool kW4>
+// Accumulator set and phase parity used by segment q.
+__device__ __forceinline__ void acc_slot(const GemmParams& p, int q, int& buf, uint32_t& parity) {
+  buf = p.nbuf == 2 ? (q & 1) : 0;
+  parity = static_cast<uint32_t>(p.nbuf == 2 ? (q >> 1) : q) & 1u;
+}
+
+// KS: 64-wide k-blocks per pipeline stage.  MT: 128-row weight sub-tiles per
+// output tile (MT = 2 lets two M = 128 MMAs share every activation tile, which
+// halves the activation bytes each CTA pulls from L2 per unit of work).
+// kTS: the dequantized A tiles go to tensor memory (tcgen05.st) instead of
+// shared memory and the MMA reads A from there, which frees shared memory for
+// a deeper load ring and allows a deep A ring beside the accumulators.
+template <bool kW4, int KS, int MT, bool kTS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                    const GemmParams p) {
+  static_assert(kW4 || MT == 1, "fp16 weights use one M sub-tile");
+  static_assert(!kTS || (kW4 && KS == 1 && MT == 1), "tensor-memory A: 4-bit weights, one k-block, one sub-tile");
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  // Every ring slot holds one k-step.
   const int SL = p.load_stages, SA = p.a_stages;
-  uint8_t* a_ring = smem;                     // SA x 16 KB (4-bit weights only)
-  uint8_t* l_ring = smem + SA * kATileBytes;  // SL x load_stage_bytes
+  constexpr uint32_t a_slot_bytes = KS * MT * kATileBytes;
+  uint8_t* a_ring = smem;                       // SA x [KS][MT] fp16 A tiles (4-bit weights only)
+  uint8_t* l_ring = smem + (kTS ? 0 : SA * a_slot_bytes);  // SL x load_stage_bytes
   uint64_t* full = reinterpret_cast<uint64_t*>(l_ring + SL * p.load_stage_bytes);
   uint64_t* empty = full + SL;
   uint64_t* afull = empty + SL;
@@ -266,14 +306,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = abort_flag + 1;
+  volatile int* fin_count = abort_flag + 2;
+  int* fin_slots = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + kBarrierBytes / 2);  // [kMaxContrib]
   float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + kBarrierBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;
-  // load stage layout: 4-bit = [B tile | raw chunk]; fp16 = [A tile | B tile]
-  const uint32_t b_off = kW4 ? 0u : static_cast<uint32_t>(kATileBytes);
+  const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;  // one 64-wide activation box
+  // load slot: 4-bit = [KS activation boxes | MT x KS raw chunks]; fp16 = [KS weight boxes | KS activation boxes]
+  const uint32_t b_off = kW4 ? 0u : static_cast<uint32_t>(KS * kATileBytes);
+  const uint32_t raw_off = KS * b_bytes;
+  constexpr int kTileCols = MT * 128;  // output features per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SL; ++s) {
@@ -292,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * p.tmem_cols);
+    tmem_alloc(tmem_slot, p.tmem_alloc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -314,8 +358,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool stop = false;
       for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
         const int n_tile = g.tile % sc.n_tiles;
-        const int t_tile = g.tile / sc.n_tiles;
-        for (int kb = g.kb0; kb < g.kb1; ++kb, ++i, rl.next(SL)) {
+        const int t_row = (g.tile / sc.n_tiles) * p.tok_tile;
+        const int mt_n = min(MT, p.n_sub - n_tile * MT);  // sub-tiles present in this tile
+        const uint32_t tx_bytes = kW4 ? KS * (static_cast<uint32_t>(mt_n * kTileBytes) + b_bytes)
+                                      : KS * (static_cast<uint32_t>(kATileBytes) + b_bytes);
+        const uint8_t* wsrc = p.wq + (static_cast<size_t>(n_tile) * MT * p.kb_real + g.kb0 * KS) * kTileBytes;
+        const size_t w_sub = static_cast<size_t>(p.kb_real) * kTileBytes;  // bytes per 128-row sub-tile
+        for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL), wsrc += KS * kTileBytes) {
           const int s = rl.s;
           if (!mbar_wait(&empty[s], rl.ph ^ 1u, p.wait_ns)) {
             set_error(p.err, DEV_TIMEOUT_PRODUCER);
@@ -326,15 +375,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* st = l_ring + s * p.load_stage_bytes;
+          mbar_arrive_expect_tx(&full[s], tx_bytes);
           if (kW4) {
-            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kTileBytes) + b_bytes);
-            bulk_load(st + b_bytes, p.wq + (static_cast<size_t>(n_tile) * sc.kb_total + kb) * kTileBytes,
-                      kTileBytes, &full[s], pol_w);
-          } else {
-            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kATileBytes) + b_bytes);
-            tma_load_2d(st, &tmap_w, &full[s], kb * 64, n_tile * 128, pol_w);
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+              if (mt < mt_n) bulk_load(st + raw_off + mt * KS * kTileBytes, wsrc + mt * w_sub, KS * kTileBytes, &full[s], pol_w);
           }
-          tma_load_2d(st + b_off, &tmap_x, &full[s], kb * 64, t_tile * p.tok_tile, pol_x);
+#pragma unroll
+          for (int u = 0; u < KS; ++u) {
+            const int kx = (ks * KS + u) * 64;
+            if (!kW4) tma_load_2d(st + u * kATileBytes, &tmap_w, &full[s], kx, n_tile * 128, pol_w);
+            tma_load_2d(st + b_off + u * b_bytes, &tmap_x, &full[s], kx, t_row, pol_x);
+          }
         }
       }
       // Never leave the CTA with bulk copies still landing in its shared memory.
@@ -345,19 +397,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
+      // descriptors of slot 0; a slot is reached by adding its byte offset >> 4
+      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(kW4 ? a_ring : l_ring));
+      const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(l_ring + b_off));
+      const uint32_t a_step = (kW4 ? a_slot_bytes : p.load_stage_bytes) >> 4;
+      const uint32_t l_step = p.load_stage_bytes >> 4;
       Ring rl, ra;
       Seg g;
       bool stop = false;
       for (int q = 0; get_seg(sc, cta, q, g); ++q) {
-        const int buf = q & 1;
-        if (!stop && !mbar_wait(&acce[buf], (static_cast<uint32_t>(q >> 1) & 1u) ^ 1u, p.wait_ns)) {
+        int buf;
+        uint32_t par;
+        acc_slot(p, q, buf, par);
+        if (!stop && !mbar_wait(&acce[buf], par ^ 1u, p.wait_ns)) {
           set_error(p.err, DEV_TIMEOUT_MMA);
           *abort_flag = 1;
         }
         if (*abort_flag) stop = true;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.tmem_cols;
-        for (int kb = g.kb0; kb < g.kb1 && !stop; ++kb, rl.next(SL), ra.next(SA)) {
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols;
+        const int mt_n = min(MT, p.n_sub - (g.tile % sc.n_tiles) * MT);
+        for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, rl.next(SL), ra.next(SA)) {
           const int s = rl.s;
           const int sa = kW4 ? ra.s : 0;
           const bool ok = kW4 ? mbar_wait(&afull[sa], ra.ph, p.wait_ns) : mbar_wait(&full[s], rl.ph, p.wait_ns);
@@ -369,13 +429,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          tc_fence_after();
-          uint8_t* st = l_ring + s * p.load_stage_bytes;
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(kW4 ? a_ring + sa * kATileBytes : st));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(st + b_off));
+          const uint64_t adesc = adesc0 + static_cast<uint64_t>((kW4 ? sa : s) * a_step);
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * l_step);
+          if (kTS) {
+            tc_fence_after();
+            const uint32_t a_tmem = tmem_base + p.a_col0 + static_cast<uint32_t>(sa) * 32u;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > g.kb0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (ks > g.kb0 || kk > 0) ? 1u : 0u);
+          } else
+#pragma unroll
+          for (int u = 0; u < KS; ++u)
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+              if (mt < mt_n) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_f16_ss(d_tmem + mt * p.m_stride, adesc + (u * MT + mt) * (kATileBytes >> 4) + 2 * kk,
+                             bdesc + u * (b_bytes >> 4) + 2 * kk, idesc, (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
+              }
           mma_commit(&empty[s]);
           if (kW4) mma_commit(&aempty[sa]);
         }
@@ -386,7 +458,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ dequantize
-    if (kW4) {
+    if (kTS) {
+      // Warp w owns TMEM lanes 32*(w%4).. (the rows it may store to) and one
+      // 32-wide half of each k-block; each thread dequantizes one row's half.
+      const int quarter = warp & 3;
+      const int hf = (warp - 2) >> 2;
+      const int row = quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + p.a_col0 + hf * 16;
+      Ring rl, ra;
+      Seg g;
+      bool stop = false;
+      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
+        for (int ks = g.kb0; ks < g.kb1; ++ks, rl.next(SL), ra.next(SA)) {
+          const int s = rl.s;
+          const int sa = ra.s;
+          bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
+          ok = ok && mbar_wait(&aempty[sa], ra.ph ^ 1u, p.wait_ns);
+          if (!ok) {
+            set_error(p.err, DEV_TIMEOUT_CONSUMER);
+            *abort_flag = 1;
+          }
+          // tcgen05.st is warp-collective: the whole warp stops or none of it
+          if (__any_sync(0xffffffffu, !ok || *abort_flag != 0)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* raw = l_ring + s * p.load_stage_bytes + raw_off;
+          const uint4 c = *reinterpret_cast<const uint4*>(raw + row * 32 + hf * 16);
+          const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
+          const __half2 m2 = __low2half2(mm);
+          const __half2 s2 = __high2half2(mm);
+          const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+          uint32_t r[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 d = dequant8(words[j], s2, m2);
+            r[4 * j] = d.x;
+            r[4 * j + 1] = d.y;
+            r[4 * j + 2] = d.z;
+            r[4 * j + 3] = d.w;
+          }
+          tmem_st_x16(t_row + static_cast<uint32_t>(sa) * 32u, r);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&afull[sa]);
+        }
+      }
+    } else if (kW4) {
       const int ct = threadIdx.x - 64;
       const int row = ct >> 1;
       const int hf = ct & 1;
@@ -394,7 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       Seg g;
       bool stop = false;
       for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-        for (int kb = g.kb0; kb < g.kb1; ++kb, rl.next(SL), ra.next(SA)) {
+        const int mt_n = min(MT, p.n_sub - (g.tile % sc.n_tiles) * MT);
+        for (int ks = g.kb0; ks < g.kb1; ++ks, rl.next(SL), ra.next(SA)) {
           const int s = rl.s;
           const int sa = ra.s;
           bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
@@ -407,18 +527,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          const uint8_t* raw = l_ring + s * p.load_stage_bytes + b_bytes;
-          const uint4 c = *reinterpret_cast<const uint4*>(raw + row * 32 + hf * 16);
-          const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
-          const __half2 m2 = __low2half2(mm);
-          const __half2 s2 = __high2half2(mm);
-          uint8_t* arow = a_ring + sa * kATileBytes + row * 128;
-          const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+          const uint8_t* raw = l_ring + s * p.load_stage_bytes + raw_off;
+          uint4 c[MT][KS];
+          __half2 mm[MT][KS];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int phys = (hf * 4 + j) ^ (row & 7);
-            *reinterpret_cast<uint4*>(arow + phys * 16) = dequant8(words[j], s2, m2);
-          }
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int u = 0; u < KS; ++u) {
+              const uint8_t* chunk = raw + (mt * KS + u) * kTileBytes;
+              if (mt < mt_n) {
+                c[mt][u] = *reinterpret_cast<const uint4*>(chunk + row * 32 + hf * 16);
+                mm[mt][u] = *reinterpret_cast<const __half2*>(chunk + kTileCodeBytes + row * 4);
+              }
+            }
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int u = 0; u < KS; ++u) {
+              if (mt >= mt_n) continue;
+              const __half2 m2 = __low2half2(mm[mt][u]);
+              const __half2 s2 = __high2half2(mm[mt][u]);
+              uint8_t* arow = a_ring + sa * a_slot_bytes + (u * MT + mt) * kATileBytes + row * 128;
+              const uint32_t words[4] = {c[mt][u].x, c[mt][u].y, c[mt][u].z, c[mt][u].w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int phys = (hf * 4 + j) ^ (row & 7);
+                *reinterpret_cast<uint4*>(arow + phys * 16) = dequant8(words[j], s2, m2);
+              }
+            }
           fence_proxy_async_smem();
           mbar_arrive(&afull[sa]);
         }
@@ -430,42 +566,47 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qd = warp & 3;  // TMEM lane quarter this warp may access
     Seg g;
     for (int q = 0; get_seg(sc, cta, q, g); ++q) {
-      const int buf = q & 1;
-      const bool ok = mbar_wait(&accf[buf], static_cast<uint32_t>(q >> 1) & 1u, drain_ns(p.wait_ns));
+      int buf;
+      uint32_t par;
+      acc_slot(p, q, buf, par);
+      const bool ok = mbar_wait(&accf[buf], par, drain_ns(p.wait_ns));
       if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
       tc_fence_after();
-      const bool aborted = !ok || *abort_flag;
+      const bool aborted = epi_any(!ok || *abort_flag);
       const int n_tile = g.tile % sc.n_tiles;
       const int t_tile = g.tile / sc.n_tiles;
-      const int frow = qd * 32 + lane;  // feature row inside the tile
       float* stg = epi_stage + (warp - kEpiWarp0) * 16 * 33;
       const int tok0 = t_tile * p.tok_tile;
-      const uint32_t tbase = tmem_base + static_cast<uint32_t>(buf) * p.tmem_cols +
-                             (static_cast<uint32_t>(qd * 32) << 16);
-      float* slot = g.full ? nullptr : p.partials + static_cast<size_t>(g.slot) * p.tok_tile * 128;
-      for (int c0 = 0; c0 < p.tok_tile && !aborted; c0 += 16) {
-        uint32_t rr[16];
-        tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
-        tmem_ld_wait();
-        if (slot) {
+      float* slot = g.full ? nullptr : p.partials + static_cast<size_t>(g.slot) * p.tok_tile * kTileCols;
+#pragma unroll 1
+      for (int mt = 0; mt < MT && !aborted; ++mt) {
+        const int frow = mt * 128 + qd * 32 + lane;  // feature row inside the tile
+        const uint32_t tbase = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + mt * p.m_stride +
+                               (static_cast<uint32_t>(qd * 32) << 16);
+        for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
+          uint32_t rr[16];
+          tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
+          tmem_ld_wait();
+          if (slot) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) slot[(c0 + j) * 128 + frow] = __uint_as_float(rr[j]);
-        } else {
-          // transpose 32 features x 16 tokens through shared memory so each
-          // lane finishes 16 consecutive features of one token
+            for (int j = 0; j < 16; ++j) slot[(c0 + j) * kTileCols + frow] = __uint_as_float(rr[j]);
+          } else {
+            // transpose 32 features x 16 tokens through shared memory so each
+            // lane finishes 16 consecutive features of one token
 #pragma unroll
-          for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = __uint_as_float(rr[j]);
-          __syncwarp();
-          const int jt = lane >> 1, hf = lane & 1;
-          const int tok = tok0 + c0 + jt;
-          const int f0 = n_tile * 128 + qd * 32 + hf * 16;
-          if (tok < p.m && f0 < p.n) {
-            float v[16];
+            for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = __uint_as_float(rr[j]);
+            __syncwarp();
+            const int jt = lane >> 1, hf = lane & 1;
+            const int tok = tok0 + c0 + jt;
+            const int f0 = n_tile * kTileCols + mt * 128 + qd * 32 + hf * 16;
+            if (tok < p.m && f0 < p.n) {
+              float v[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] = stg[jt * 33 + hf * 16 + u];
-            store_row16(p, v, tok, f0);
+              for (int u = 0; u < 16; ++u) v[u] = stg[jt * 33 + hf * 16 + u];
+              store_row16(p, v, tok, f0);
+            }
+            __syncwarp();
           }
-          __syncwarp();
         }
       }
       tc_fence_before();
@@ -475,80 +616,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       epi_bar();
       if (et == 0) {
-        int ncontrib;
+        int ns = 0;
         if (sc.mode == SCHED_SPLITS) {
-          ncontrib = sc.splits;
+          for (int part = 0; part < sc.splits && ns < kMaxContrib; ++part) fin_slots[ns++] = g.tile * sc.splits + part;
         } else {
           const long long t0 = static_cast<long long>(g.tile) * sc.kb_total;
-          const int lo = sk_first_contributor(sc, t0);
-          int hi = lo;
-          while (hi + 1 < sc.grid && sk_start(sc, hi + 1) < t0 + sc.kb_total) ++hi;
-          ncontrib = hi - lo + 1;
+          for (int c = sk_first_contributor(sc, t0); c < sc.grid && sk_start(sc, c) < t0 + sc.kb_total &&
+                                                     ns < kMaxContrib;
+               ++c)
+            fin_slots[ns++] = 2 * c + (sk_start(sc, c) >= t0 ? 0 : 1);
         }
+        *fin_count = ns;
         const int old = atomicAdd(&p.counters[g.tile], 1);
-        *last_flag = old == ncontrib - 1;
+        *last_flag = old == ns - 1;
       }
       epi_bar();
       const bool last = *last_flag;
-      epi_bar();  // everyone has read the flag before it can be rewritten
-      if (!last) continue;
-      __threadfence();
-      int slots[kMaxContrib];
-      int ns = 0;
-      if (sc.mode == SCHED_SPLITS) {
-        for (int part = 0; part < sc.splits && ns < kMaxContrib; ++part) slots[ns++] = g.tile * sc.splits + part;
-      } else {
-        const long long t0 = static_cast<long long>(g.tile) * sc.kb_total;
-        for (int c = sk_first_contributor(sc, t0); c < sc.grid && sk_start(sc, c) < t0 + sc.kb_total &&
-                                                   ns < kMaxContrib;
-             ++c)
-          slots[ns++] = 2 * c + (sk_start(sc, c) >= t0 ? 0 : 1);
-      }
-      // Sum the slots in contributor order with coalesced 16-byte loads (two
-      // contributors in flight): thread et finishes features 16*(et%8)..+15 of
-      // tokens et/8, et/8 + 16, ... of the tile.
-      const int fg = (et & 7) * 16;
-      const int tsub = et >> 3;
-      const int f0 = n_tile * 128 + fg;
-      for (int c = tsub; c < p.tok_tile; c += 16) {
-        float acc[16];
+      const int ns = *fin_count;
+      if (last) {
+        __threadfence();
+        // Sum the slots in contributor order with coalesced 16-byte loads (two
+        // contributors in flight): thread et finishes 16 consecutive features
+        // of tokens et/8, et/8 + 16, ... for each 128-feature sub-tile.
+        const int tsub = et >> 3;
+        for (int mt = 0; mt < MT; ++mt) {
+          const int fg = mt * 128 + (et & 7) * 16;
+          const int f0 = n_tile * kTileCols + fg;
+          for (int c = tsub; c < p.tok_tile; c += 16) {
+            float acc[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) acc[u] = 0.f;
-        int k = 0;
-        for (; k + 1 < ns; k += 2) {
-          const float4* b0 = reinterpret_cast<const float4*>(
-              p.partials + (static_cast<size_t>(slots[k]) * p.tok_tile + c) * 128 + fg);
-          const float4* b1 = reinterpret_cast<const float4*>(
-              p.partials + (static_cast<size_t>(slots[k + 1]) * p.tok_tile + c) * 128 + fg);
-          float4 v0[4], v1[4];
+            for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+            int k = 0;
+            for (; k + 1 < ns; k += 2) {
+              const float4* b0 = reinterpret_cast<const float4*>(
+                  p.partials + (static_cast<size_t>(fin_slots[k]) * p.tok_tile + c) * kTileCols + fg);
+              const float4* b1 = reinterpret_cast<const float4*>(
+                  p.partials + (static_cast<size_t>(fin_slots[k + 1]) * p.tok_tile + c) * kTileCols + fg);
+              float4 v0[4], v1[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            v0[u] = __ldcg(b0 + u);
-            v1[u] = __ldcg(b1 + u);
-          }
+              for (int u = 0; u < 4; ++u) {
+                v0[u] = __ldcg(b0 + u);
+                v1[u] = __ldcg(b1 + u);
+              }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            acc[4 * u] += v0[u].x + v1[u].x;
-            acc[4 * u + 1] += v0[u].y + v1[u].y;
-            acc[4 * u + 2] += v0[u].z + v1[u].z;
-            acc[4 * u + 3] += v0[u].w + v1[u].w;
-          }
-        }
-        if (k < ns) {
-          const float4* b0 = reinterpret_cast<const float4*>(
-              p.partials + (static_cast<size_t>(slots[k]) * p.tok_tile + c) * 128 + fg);
+              for (int u = 0; u < 4; ++u) {
+                acc[4 * u] += v0[u].x + v1[u].x;
+                acc[4 * u + 1] += v0[u].y + v1[u].y;
+                acc[4 * u + 2] += v0[u].z + v1[u].z;
+                acc[4 * u + 3] += v0[u].w + v1[u].w;
+              }
+            }
+            if (k < ns) {
+              const float4* b0 = reinterpret_cast<const float4*>(
+                  p.partials + (static_cast<size_t>(fin_slots[k]) * p.tok_tile + c) * kTileCols + fg);
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float4 v = __ldcg(b0 + u);
-            acc[4 * u] += v.x;
-            acc[4 * u + 1] += v.y;
-            acc[4 * u + 2] += v.z;
-            acc[4 * u + 3] += v.w;
+              for (int u = 0; u < 4; ++u) {
+                const float4 v = __ldcg(b0 + u);
+                acc[4 * u] += v.x;
+                acc[4 * u + 1] += v.y;
+                acc[4 * u + 2] += v.z;
+                acc[4 * u + 3] += v.w;
+              }
+            }
+            const int tok = tok0 + c;
+            if (tok < p.m && f0 < p.n) store_row16(p, acc, tok, f0);
           }
         }
-        const int tok = tok0 + c;
-        if (tok < p.m && f0 < p.n) store_row16(p, acc, tok, f0);
       }
+      epi_bar();  // everyone is done with the flag and the slot list before they are rewritten
     }
   }
   tc_fence_before();
@@ -560,11 +695,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       Seg g;
       int nq = 0;
       while (get_seg(sc, cta, nq, g)) ++nq;
-      if (nq > 0) mbar_wait(&accf[(nq - 1) & 1], static_cast<uint32_t>((nq - 1) >> 1) & 1u, drain_ns(p.wait_ns));
+      if (nq > 0) {
+        int buf;
+        uint32_t par;
+        acc_slot(p, nq - 1, buf, par);
+        mbar_wait(&accf[buf], par, drain_ns(p.wait_ns));
+      }
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * p.tmem_cols);
+    tmem_dealloc(tmem_base, p.tmem_alloc);
   }
 }
 
@@ -605,9 +745,15 @@ bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, i
 
 struct Plan {
   int tok_tile, tok_tiles, n_tiles;
+  int ks;  // 64-wide k-blocks per pipeline stage
+  int mt;  // 128-row weight sub-tiles per output tile
+  bool ts;  // A (dequantized weights) in tensor memory
+  uint32_t a_col0;
   Sched sc;
   int load_stages, a_stages;
   uint32_t load_stage_bytes;
+  uint32_t acc_cols, m_stride, tmem_alloc;
+  int nbuf;
   size_t smem;
   size_t partial_bytes, counter_bytes;
 };
@@ -617,7 +763,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_tile) {
   Plan P{};
-  const int kb_total = k / 64;
+  const int kb_real = k / 64;
   if (force_tok_tile > 0) {
     P.tok_tile = force_tok_tile;
     P.tok_tiles = (m + P.tok_tile - 1) / P.tok_tile;
@@ -628,7 +774,17 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.tok_tiles = (m + 255) / 256;
     P.tok_tile = round_up((m + P.tok_tiles - 1) / P.tok_tiles, 16);
   }
-  P.n_tiles = (n + 127) / 128;
+  // Decode-sized token tiles on 4-bit weights: two 128-row sub-tiles share
+  // each activation tile (half the L2 -> SM activation traffic per MMA), or,
+  // for a single sub-tile, two k-blocks per stage (half the hand-offs).
+  const bool decode_w4 = w_bits == 4 && P.tok_tile <= 160;
+  P.ts = false;  // measured slower than two k-blocks per shared-memory stage
+  P.mt = 1;
+  P.ks = decode_w4 && !P.ts && kb_real % 2 == 0 ? 2 : 1;
+  const int kb_total = kb_real / P.ks;  // k-steps per tile
+  const int min_iters = max(1, kMinItersPerCta / (P.ks * P.mt));
+  const int n_sub = (n + 127) / 128;
+  P.n_tiles = (n_sub + P.mt - 1) / P.mt;
   const int tiles = P.n_tiles * P.tok_tiles;
   const int sms = runtime().num_sms;
   Sched& s = P.sc;
@@ -638,7 +794,7 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   s.iters = static_cast<long long>(tiles) * kb_total;
   s.splits = 1;
   s.per = kb_total;
-  const size_t tile_bytes = static_cast<size_t>(P.tok_tile) * 128 * sizeof(float);
+  const size_t tile_bytes = static_cast<size_t>(P.tok_tile) * P.mt * 128 * sizeof(float);
   if (force_splits > 1) {
     s.mode = SCHED_SPLITS;
     s.per = (kb_total + force_splits - 1) / force_splits;
@@ -648,13 +804,13 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     if (s.splits > 1) P.partial_bytes = static_cast<size_t>(s.grid) * tile_bytes;
     else s.mode = SCHED_TILES, s.grid = min(tiles, sms);
   } else if (force_splits == 1 || tiles >= 16 * sms ||
-             tiles % std::max<long long>(1, std::min<long long>(sms, s.iters / kMinItersPerCta)) == 0) {
+             tiles % std::max<long long>(1, std::min<long long>(sms, s.iters / min_iters)) == 0) {
     // many tiles, or whole tiles already divide evenly over the CTAs stream-K would use
     s.mode = SCHED_TILES;
     s.grid = min(tiles, sms);
   } else {
     s.mode = SCHED_STREAMK;
-    s.grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, s.iters / kMinItersPerCta)));
+    s.grid = static_cast<int>(std::min<long long>(sms, std::max<long long>(1, s.iters / min_iters)));
     // A tile is shared by at most ceil(kb_total / (iters / grid)) + 1 CTAs.
     const long long per_cta = s.iters / s.grid;
     if ((kb_total + per_cta - 1) / per_cta + 1 > kMaxContrib)
@@ -662,30 +818,64 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.partial_bytes = static_cast<size_t>(2) * s.grid * tile_bytes;
   }
   if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * sizeof(int);
+  // TMEM: one accumulator set = mt sub-tiles x tok_tile fp32 columns; two sets
+  // when they fit in the 512 columns, so the epilogue overlaps the next segment.
+  P.m_stride = static_cast<uint32_t>(P.mt == 1 ? P.tok_tile : round_up(P.tok_tile, 32));
+  const uint32_t set = P.mt == 1 ? P.m_stride : P.mt * P.m_stride;
+  uint32_t set_pow2 = 32;
+  while (set_pow2 < set) set_pow2 <<= 1;
+  if (P.mt == 1) {
+    P.acc_cols = set_pow2;  // power-of-two sets
+    P.nbuf = 2;
+  } else {
+    P.acc_cols = set;
+    P.nbuf = 2 * set <= 512 ? 2 : 1;
+  }
+  if (P.ts) {
+    // two accumulator sets, then the A ring: 32 columns (128 x 64 fp16) per stage
+    P.acc_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
+    P.nbuf = 2;
+    P.a_col0 = 2 * P.acc_cols;
+  }
+  P.tmem_alloc = P.ts ? 512 : 32;
+  while (P.tmem_alloc < P.nbuf * P.acc_cols) P.tmem_alloc <<= 1;
   const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
-  if (w_bits == 4) {
-    P.a_stages = P.tok_tile > 128 && P.tok_tile != 144 ? 2 : 3;
-    P.load_stage_bytes = static_cast<uint32_t>(P.tok_tile * 128 + kRawBytes);
-    P.load_stages = min(kMaxLoadStages, static_cast<int>((budget - P.a_stages * kATileBytes) / P.load_stage_bytes));
+  const int b_bytes = P.tok_tile * 128;
+  int a_slot = 0;
+  if (P.ts) {
+    P.a_stages = min(8, static_cast<int>((512 - P.a_col0) / 32));
+    P.load_stage_bytes = static_cast<uint32_t>(b_bytes + round_up(kTileBytes, 1024));
+  } else if (w_bits == 4) {
+    a_slot = P.ks * P.mt * kATileBytes;
+    P.a_stages = P.mt == 2 ? 3 : (P.ks == 2 ? 2 : (P.tok_tile > 128 && P.tok_tile != 144 ? 2 : 3));
+    P.load_stage_bytes = static_cast<uint32_t>(P.ks * b_bytes + round_up(P.mt * P.ks * kTileBytes, 1024));
   } else {
     P.a_stages = 0;
-    P.load_stage_bytes = static_cast<uint32_t>(kATileBytes + P.tok_tile * 128);
-    P.load_stages = min(kMaxLoadStages, static_cast<int>(budget / P.load_stage_bytes));
+    P.load_stage_bytes = static_cast<uint32_t>(P.ks * (kATileBytes + b_bytes));
   }
-  P.load_stages = min(P.load_stages, static_cast<int>((budget - P.a_stages * kATileBytes) / P.load_stage_bytes));
-  P.smem = static_cast<size_t>(P.a_stages) * kATileBytes + static_cast<size_t>(P.load_stages) * P.load_stage_bytes +
+  P.load_stages = min(kMaxLoadStages, (budget - P.a_stages * a_slot) / static_cast<int>(P.load_stage_bytes));
+  P.smem = static_cast<size_t>(P.a_stages) * a_slot + static_cast<size_t>(P.load_stages) * P.load_stage_bytes +
            1024 + kBarrierBytes + kEpiStageBytes;
   return P;
 }
 
-template <bool kW4>
+template <bool kW4, int KS, int MT, bool kTS>
 cudaError_t configure_once() {
   static cudaError_t status = cudaErrorNotReady;
   static std::once_flag once;
   std::call_once(once, [] {
-    status = cudaFuncSetAttribute(gemm_tc_kernel<kW4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    status = cudaFuncSetAttribute(gemm_tc_kernel<kW4, KS, MT, kTS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   });
   return status;
+}
+
+template <bool kW4, int KS, int MT, bool kTS = false>
+cudaError_t launch_variant(const Plan& P, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
+                           cudaStream_t s) {
+  const cudaError_t e = configure_once<kW4, KS, MT, kTS>();
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<kW4, KS, MT, kTS><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
+  return launched();
 }
 
 }  // namespace
@@ -701,8 +891,7 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   const Plan P = make_plan(a.m, a.n, a.k, a.w_bits, a.force_splits, a.force_tok_tile);
   const bool w4 = a.w_bits == 4;
   if (P.load_stages < 2) return cudaErrorInvalidValue;
-  cudaError_t e = w4 ? configure_once<true>() : configure_once<false>();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
   CUtensorMap tx, tw;
   if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile)) return cudaErrorInvalidValue;
   if (w4) {
@@ -716,12 +905,16 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.n = a.n;
   p.k = a.k;
   p.tok_tile = P.tok_tile;
+  p.kb_real = a.k / 64;
   p.load_stages = P.load_stages;
   p.a_stages = P.a_stages;
   p.load_stage_bytes = P.load_stage_bytes;
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
-  p.tmem_cols = cols;
+  p.n_sub = (a.n + 127) / 128;
+  p.acc_cols = P.acc_cols;
+  p.m_stride = P.m_stride;
+  p.tmem_alloc = P.tmem_alloc;
+  p.nbuf = P.nbuf;
+  p.a_col0 = P.a_col0;
   p.sc = P.sc;
   p.bias = a.bias;
   p.residual = a.residual;
@@ -744,11 +937,11 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
     e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  if (w4)
-    gemm_tc_kernel<true><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
-  else
-    gemm_tc_kernel<false><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
-  return launched();
+  if (w4 && P.ts) return launch_variant<true, 1, 1, true>(P, tx, tw, p, s);
+  if (w4 && P.mt == 2) return launch_variant<true, 1, 2>(P, tx, tw, p, s);
+  if (w4 && P.ks == 2) return launch_variant<true, 2, 1>(P, tx, tw, p, s);
+  if (w4) return launch_variant<true, 1, 1>(P, tx, tw, p, s);
+  return launch_variant<false, 1, 1>(P, tx, tw, p, s);
 }
 
 }  // namespace flexq

@@ -83,11 +83,23 @@ __global__ void kv_append_v4_tokens_kernel(const __half* __restrict__ src, int l
   uint32_t* w = words + (head_row * (kv_pad_len(max_len) / 8) + slot / 8) * d + gd * 64 + half_id * 32;
   const int sh = 4 * (slot & 7);
   const uint32_t clear = ~(0xFu << sh);
+  if (exclusive) {
+    // the lane owns these 32 words: one 128-byte read-modify-write in 16-byte vectors
+    uint4* w4 = reinterpret_cast<uint4*>(w);
+    uint4 cur[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cur[u] = w4[u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cur[u].x = (cur[u].x & clear) | (q[4 * u] << sh);
+      cur[u].y = (cur[u].y & clear) | (q[4 * u + 1] << sh);
+      cur[u].z = (cur[u].z & clear) | (q[4 * u + 2] << sh);
+      cur[u].w = (cur[u].w & clear) | (q[4 * u + 3] << sh);
+      w4[u] = cur[u];
+    }
+  } else {
 #pragma unroll 4
-  for (int e = 0; e < 32; ++e) {
-    if (exclusive) {
-      w[e] = (w[e] & clear) | (q[e] << sh);
-    } else {
+    for (int e = 0; e < 32; ++e) {
       atomicAnd(w + e, clear);
       atomicOr(w + e, q[e] << sh);
     }

@@ -46,7 +46,7 @@ def test_static_scratch_matches_workspace_linear_twice(m, n, k, splits):
 
 
 def test_static_scratch_rejects_oversized_split():
-    m, n, k = 300, 8192, 128
+    m, n, k = 600, 8192, 128  # 3 token tiles of 208, 64 feature tiles, 2 K-splits: ~40 MB
     x = torch.zeros(m, k, dtype=torch.float16, device="cuda")
     wq = torch.zeros(fq.flexq_packed_weight_bytes(n, k), dtype=torch.uint8, device="cuda")
     y = torch.zeros(m, n, dtype=torch.float16, device="cuda")
