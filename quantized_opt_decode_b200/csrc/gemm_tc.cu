@@ -11,32 +11,53 @@
 //
 // One output tile = 128 features x up to 256 tokens; the weight is the MMA's A
 // operand, so a small decode batch becomes the MMA's N.  A persistent CTA per
-// SM walks a list of (tile, k-block range) segments:
-//   warp 0      TMA producer: per k-step (one or two 64-wide k-blocks) one
-//               cp.async.bulk of the packed 4-bit chunks (codes + min/scale,
-//               4608 contiguous bytes per k-block) or tiled fp16 weight
-//               boxes, plus 128-byte-swizzled cp.async.bulk.tensor boxes of
-//               the activations, into a deep ring;
-//   warps 2-9   dequantize the chunk into a short ring of fp16 A tiles in the
-//               UMMA K-major SW128 layout ((code | 0x6400) is the fp16 value
-//               1024 + code; one half2 subtract and one half2 fused
-//               multiply-add give code * scale + min rounded once);
-//   warp 1      owns TMEM (two accumulator buffers) and, from one thread,
-//               issues tcgen05.mma.kind::f16 (M=128, N=tokens, K=16) x 4 per
-//               k-block, releasing ring slots with tcgen05.commit;
-// Each mbarrier hand-off costs a few hundred cycles of latency in these
-// scalar role loops, so decode-sized tiles on 4-bit weights move two k-blocks
-// per stage (half the hand-offs per tile).
-//   warps 10-13 epilogue: tcgen05.ld, + bias, GELU, + residual, fp16 or fp32
-//               store; overlaps the next segment's main loop.
+// SM walks a list of (tile, k-block range) segments.  Two kernels share the
+// scheduler and the epilogue:
+//
+// gemm_w4_decode_kernel (4-bit weights, decode-sized token tiles <= 160 whose K
+// has an odd number of 64-wide k-blocks):
+//   warp 0      TMA producer: per 64-wide k-block one cp.async.bulk of the
+//               packed chunk (codes + min/scale, 4608 contiguous bytes) and
+//               one 128-byte-swizzled cp.async.bulk.tensor of the activations
+//               into a deep shared-memory ring;
+//   warps 2-9   two dequantizing warpgroups taking alternate k-blocks.  Each
+//               thread turns one weight row of the k-block into fp16
+//               ((code | 0x6400) is the fp16 value 1024 + code; one half2
+//               subtract and one half2 fused multiply-add give
+//               code * scale + min rounded once) and stores it straight into
+//               tensor memory (tcgen05.st): no shared-memory round trip for
+//               A.  A named barrier closes the group's step and one thread
+//               signals it with a single mbarrier arrival.  Each group has
+//               its own A ring in tensor memory, so the two groups' steps
+//               overlap;
+//   warp 1      owns TMEM and, from one thread, issues the k-blocks'
+//               tcgen05.mma.kind::f16 (M=128, N=tokens, K=16, A from tensor
+//               memory) x 4 in k order, alternating between the groups' rings.
+//               The issuing thread stalls while the tensor pipe's queue is
+//               full; keeping it out of the dequantizing warps keeps that
+//               stall off their critical path;
+//   warps 10-13 epilogue (below).
+//
+// gemm_tc_kernel (everything else: prefill-sized tiles, fp16 weights, and
+// decode-sized 4-bit tiles with an even number of k-blocks, which it moves two
+// k-blocks per pipeline stage; on the OPT-30B decode shapes this measured
+// faster than the tensor-memory-A kernel):
+//   warp 0 TMA producer; warps 2-9 dequantize into a shared-memory ring of
+//   fp16 A tiles in the UMMA K-major SW128 layout; warp 1 issues the MMAs from
+//   one thread (A and B from shared memory); warps 10-13 epilogue.
+//
+// Epilogue (warps 10-13, one TMEM lane quarter each): tcgen05.ld, + bias,
+// GELU, + residual, fp16 or fp32 store; two accumulator buffers let it overlap
+// the next segment's main loop.
 // Scheduling: whole tiles round-robin over the SMs when there are many; when
 // the grid is small (decode), each SM takes an equal share of all k-blocks
-// (stream-K, in units of k-steps), so tiles may be split across CTAs.  A partial tile is written
-// to a per-contributor fp32 slot; the contributor that arrives last (an atomic
-// counter per tile) sums the slots in contributor order and applies the
+// (stream-K), so tiles may be split across CTAs.  Every contributor of a split
+// tile counts itself in; the one that arrives last does not write its own
+// partial: it waits until the others' fp32 partials are published, then sums
+// them and its own accumulator (in TMEM) in contributor order and applies the
 // epilogue, so results do not depend on timing.
-// Every mbarrier wait is bounded; on expiry the CTA records an error code in
-// the device error word and unwinds (no trap).
+// Every wait is bounded; on expiry the CTA records an error code in the device
+// error word and unwinds (no trap).
 #include <math.h>
 
 #include <mutex>
@@ -49,15 +70,19 @@ namespace {
 
 constexpr int kThreads = 448;
 constexpr int kDequantThreads = 256;
+constexpr int kGroupThreads = 128;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
 constexpr int kATileBytes = 128 * 64 * 2;
+constexpr int kRawStageBytes = (kTileBytes + 1023) / 1024 * 1024;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
+constexpr int kMaxBarriers = 56;     // mbarriers fit in the first 448 bytes of that region
 constexpr int kEpiStageBytes = 4 * 16 * 33 * 4;  // per epilogue warp: 16 tokens x 33 floats
 constexpr int kMaxLoadStages = 16;
 constexpr int kMinItersPerCta = 8;
 constexpr int kMaxContrib = 64;
+constexpr int kDecodeMaxTok = 160;
 
 enum SchedMode : int { SCHED_TILES = 0, SCHED_STREAMK = 1, SCHED_SPLITS = 2 };
 
@@ -66,7 +91,7 @@ struct Sched {
   int grid;
   int tiles;        // n_tiles * tok_tiles
   int n_tiles;
-  int kb_total;
+  int kb_total;     // k-blocks per tile
   long long iters;  // tiles * kb_total
   int splits, per;  // SCHED_SPLITS
 };
@@ -78,12 +103,9 @@ struct GemmParams {
   int kb_real;  // 64-wide k-blocks of K
   int load_stages, a_stages;
   uint32_t load_stage_bytes;
-  int n_sub;               // 128-row weight sub-tiles (ceil(n / 128))
-  uint32_t acc_cols;       // TMEM columns of one accumulator set (all M sub-tiles)
-  uint32_t m_stride;       // TMEM column offset between M sub-tiles
-  uint32_t tmem_alloc;     // columns allocated (power of two)
-  int nbuf;                // accumulator sets (2 = epilogue overlaps the next segment)
-  uint32_t a_col0;         // first TMEM column of the A ring (tensor-memory A)
+  uint32_t acc_cols;    // TMEM columns between the two accumulator buffers
+  uint32_t tmem_alloc;  // columns allocated (power of two)
+  uint32_t a_col0;      // first TMEM column of the A rings (decode kernel)
   Sched sc;
   const __half* bias;
   const __half* residual;
@@ -94,7 +116,7 @@ struct GemmParams {
   int ldyf;
   int epi;
   float* partials;  // [slot][tok_tile][128]
-  int* counters;    // [tiles]
+  int* counters;    // [tiles][2]: contributors arrived, partials published
   uint64_t wait_ns;
   uint32_t* err;
 };
@@ -189,17 +211,18 @@ __device__ __forceinline__ uint4 dequant8(uint32_t w, __half2 s2, __half2 m2) {
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory"); }
 
-// Barrier over the epilogue threads that also ORs a predicate across them, so
-// a branch taken on it is uniform (no thread skips a later epi_bar).
-__device__ __forceinline__ bool epi_any(bool v) {
+// Named barrier over kCount threads that also ORs a predicate across them, so
+// a branch taken on the result is uniform (no thread skips a later barrier).
+template <int kCount>
+__device__ __forceinline__ bool bar_any(int id, bool v) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "n"(kEpiThreads)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "n"(kCount)
       : "memory");
   return r != 0;
 }
@@ -223,9 +246,21 @@ __device__ __forceinline__ void load_h16(const __half* src, int count, float (&v
   }
 }
 
-// Epilogue for 16 consecutive output features f0..f0+15 of one token: every
-// load is issued before any store, and full aligned rows use 16-byte vectors.
-__device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16], int tok, int f0) {
+// Bias of output features f0..f0+15 (zero where the epilogue adds none).
+__device__ __forceinline__ void load_bias16(const GemmParams& p, int f0, float (&bv)[16]) {
+  if ((p.epi & EPI_BIAS) && !(p.epi & EPI_F32_OUT) && f0 < p.n) {
+    load_h16(p.bias + f0, min(16, p.n - f0), bv);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 16; ++u) bv[u] = 0.f;
+  }
+}
+
+// Epilogue for 16 consecutive output features f0..f0+15 of one token; bv holds
+// their bias.  Every load is issued before any store, and full aligned rows
+// use 16-byte vectors.
+__device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16], const float (&bv)[16], int tok,
+                                            int f0) {
   const int count = min(16, p.n - f0);
   if (p.epi & EPI_F32_OUT) {
     float* dst = p.yf + static_cast<size_t>(tok) * p.ldyf + f0;
@@ -238,13 +273,7 @@ __device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16],
     }
     return;
   }
-  float bv[16], rv[16];
-  if (p.epi & EPI_BIAS) {
-    load_h16(p.bias + f0, count, bv);
-  } else {
-#pragma unroll
-    for (int u = 0; u < 16; ++u) bv[u] = 0.f;
-  }
+  float rv[16];
   if (p.epi & EPI_RESIDUAL) {
     load_h16(p.residual + static_cast<size_t>(tok) * p.ld_res + f0, count, rv);
   } else {
@@ -266,58 +295,451 @@ __device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16],
     reinterpret_cast<uint4*>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     reinterpret_cast<uint4*>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
   } else {
-    const __half* hv = reinterpret_cast<const __half*>(packed);
-    for (int u = 0; u < count; ++u) dst[u] = hv[u];
+#pragma unroll
+    for (int u = 0; u < 16; u += 2) {
+      if (u < count) dst[u] = __low2half(u32_as_h2(packed[u / 2]));
+      if (u + 1 < count) dst[u + 1] = __high2half(u32_as_h2(packed[u / 2]));
+    }
   }
 }
 
-// Accumulator set and phase parity used by segment q.
-__device__ __forceinline__ void acc_slot(const GemmParams& p, int q, int& buf, uint32_t& parity) {
-  buf = p.nbuf == 2 ? (q & 1) : 0;
-  parity = static_cast<uint32_t>(p.nbuf == 2 ? (q >> 1) : q) & 1u;
+// Accumulator buffer and phase parity used by segment q.
+__device__ __forceinline__ void acc_slot(int q, int& buf, uint32_t& parity) {
+  buf = q & 1;
+  parity = static_cast<uint32_t>(q >> 1) & 1u;
 }
 
-// KS: 64-wide k-blocks per pipeline stage.  MT: 128-row weight sub-tiles per
-// output tile (MT = 2 lets two M = 128 MMAs share every activation tile, which
-// halves the activation bytes each CTA pulls from L2 per unit of work).
-// kTS: the dequantized A tiles go to tensor memory (tcgen05.st) instead of
-// shared memory and the MMA reads A from there, which frees shared memory for
-// a deeper load ring and allows a deep A ring beside the accumulators.
-template <bool kW4, int KS, int MT, bool kTS>
+// Shared-memory words of the epilogue and the teardown, after the rings.
+struct Ctl {
+  uint64_t* accf;  // [2] accumulator buffer complete
+  uint64_t* acce;  // [2] accumulator buffer drained
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  volatile int* last_flag;
+  volatile int* fin_count;
+  volatile int* fin_me;
+  int* fin_slots;  // [kMaxContrib]
+  float* stage;    // [4][16][33]
+};
+
+__device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
+  Ctl c;
+  c.accf = accf;
+  c.acce = accf + 2;
+  c.tmem_slot = reinterpret_cast<uint32_t*>(region + 8 * kMaxBarriers);
+  c.abort_flag = reinterpret_cast<volatile int*>(c.tmem_slot + 1);
+  c.last_flag = c.abort_flag + 1;
+  c.fin_count = c.abort_flag + 2;
+  c.fin_me = c.abort_flag + 3;
+  c.fin_slots = reinterpret_cast<int*>(region + kBarrierBytes / 2);
+  c.stage = reinterpret_cast<float*>(region + kBarrierBytes);
+  return c;
+}
+
+// Bounded wait until a global counter reaches `target` (the other
+// contributors of a split tile have published their partials).
+__device__ __forceinline__ bool wait_counter(const int* ctr, int target, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(64);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// epilogue role (warps kEpiWarp0 .. kEpiWarp0 + 3)
+// ---------------------------------------------------------------------------
+__device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_base, int warp, int lane) {
+  const Sched& sc = p.sc;
+  const int cta = blockIdx.x;
+  const int et = threadIdx.x - kEpiWarp0 * 32;
+  const int qd = warp & 3;          // TMEM lane quarter this warp may access
+  const int frow = qd * 32 + lane;  // feature row of the tile this thread reads from TMEM
+  const int jt = lane >> 1, hf = lane & 1;
+  float* stg = c.stage + (warp - kEpiWarp0) * 16 * 33;
+  Seg g;
+  for (int q = 0; get_seg(sc, cta, q, g); ++q) {
+    int buf;
+    uint32_t par;
+    acc_slot(q, buf, par);
+    const bool ok = mbar_wait(&c.accf[buf], par, drain_ns(p.wait_ns));
+    if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
+    tc_fence_after();
+    const bool aborted = bar_any<kEpiThreads>(1, !ok || *c.abort_flag);
+    if (aborted) {
+      tc_fence_before();
+      mbar_arrive(&c.acce[buf]);
+      continue;
+    }
+    const int n_tile = g.tile % sc.n_tiles;
+    const int tok0 = (g.tile / sc.n_tiles) * p.tok_tile;
+    const uint32_t tbase =
+        tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + (static_cast<uint32_t>(qd * 32) << 16);
+    const int f_out = n_tile * 128 + qd * 32 + hf * 16;  // features this lane finishes
+    // Split tile: count in; the last to arrive finishes the tile.
+    int ns = 1, me = 0;
+    if (!g.full) {
+      if (et == 0) {
+        int n = 0, mine = 0;
+        if (sc.mode == SCHED_SPLITS) {
+          for (int part = 0; part < sc.splits && n < kMaxContrib; ++part) {
+            if (g.tile * sc.splits + part == g.slot) mine = n;
+            c.fin_slots[n++] = g.tile * sc.splits + part;
+          }
+        } else {
+          const long long t0 = static_cast<long long>(g.tile) * sc.kb_total;
+          for (int cc = sk_first_contributor(sc, t0);
+               cc < sc.grid && sk_start(sc, cc) < t0 + sc.kb_total && n < kMaxContrib; ++cc) {
+            const int sl = 2 * cc + (sk_start(sc, cc) >= t0 ? 0 : 1);
+            if (sl == g.slot) mine = n;
+            c.fin_slots[n++] = sl;
+          }
+        }
+        *c.fin_count = n;
+        *c.fin_me = mine;
+        const int old = atomicAdd(&p.counters[2 * g.tile], 1);
+        *c.last_flag = old == n - 1;
+      }
+      epi_bar();
+      const bool last = *c.last_flag;
+      ns = *c.fin_count;
+      me = *c.fin_me;
+      if (!last) {
+        // publish this contributor's fp32 partial (a warp stores 32
+        // consecutive features of one token)
+        float* slot = p.partials + static_cast<size_t>(g.slot) * p.tok_tile * 128;
+        for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
+          uint32_t rr[16];
+          __syncwarp();
+          tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) __stcg(slot + (c0 + j) * 128 + frow, __uint_as_float(rr[j]));
+        }
+        tc_fence_before();
+        mbar_arrive(&c.acce[buf]);
+        __threadfence();
+        epi_bar();
+        if (et == 0) atomicAdd(&p.counters[2 * g.tile + 1], 1);
+        continue;
+      }
+      if (et == 0 && !wait_counter(&p.counters[2 * g.tile + 1], ns - 1, drain_ns(p.wait_ns)))
+        set_error(p.err, DEV_TIMEOUT_EPILOGUE);
+      epi_bar();
+    }
+    // Finish the tile: the accumulator (plus the other contributors' partials,
+    // summed in contributor order), then bias / GELU / residual.
+    float bv[16];
+    load_bias16(p, f_out, bv);
+    const bool one_other = !g.full && ns == 2;
+    const float* other =
+        one_other ? p.partials + static_cast<size_t>(c.fin_slots[1 - me]) * p.tok_tile * 128 : nullptr;
+    float nxt[16];  // the other contributor's values for the next 16 tokens
+    if (one_other) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) nxt[j] = __ldcg(other + j * 128 + frow);
+    }
+    for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
+      uint32_t rr[16];
+      __syncwarp();
+      tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
+      float v[16];
+      if (one_other) {
+        float cur[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cur[j] = nxt[j];
+        if (c0 + 16 < p.tok_tile) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) nxt[j] = __ldcg(other + (c0 + 16 + j) * 128 + frow);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float a = __uint_as_float(rr[j]);
+          v[j] = me == 0 ? (0.f + a) + cur[j] : (0.f + cur[j]) + a;
+        }
+      } else if (!g.full) {
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.f;
+        for (int k = 0; k < ns; ++k) {
+          if (k == me) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(rr[j]);
+          } else {
+            const float* src = p.partials + static_cast<size_t>(c.fin_slots[k]) * p.tok_tile * 128;
+            float t[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) t[j] = __ldcg(src + (c0 + j) * 128 + frow);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += t[j];
+          }
+        }
+      } else {
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]);
+      }
+      // transpose 32 features x 16 tokens through shared memory so each lane
+      // finishes 16 consecutive features of one token
+#pragma unroll
+      for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = v[j];
+      __syncwarp();
+      const int tok = tok0 + c0 + jt;
+      if (tok < p.m && f_out < p.n) {
+        float o[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) o[u] = stg[jt * 33 + hf * 16 + u];
+        store_row16(p, o, bv, tok, f_out);
+      }
+      __syncwarp();
+    }
+    tc_fence_before();
+    mbar_arrive(&c.acce[buf]);
+  }
+}
+
+// Teardown shared by both kernels: free TMEM once every thread is done (the
+// MMA-issuing threads have waited for their own MMAs before getting here).
+__device__ __forceinline__ void teardown(const GemmParams& p, const Ctl& c, uint32_t tmem_base, int warp) {
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_alloc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// decode kernel: 4-bit weights, A dequantized into tensor memory by two
+// warpgroups; one thread issues the MMAs
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const GemmParams p) {
-  static_assert(kW4 || MT == 1, "fp16 weights use one M sub-tile");
-  static_assert(!kTS || (kW4 && KS == 1 && MT == 1), "tensor-memory A: 4-bit weights, one k-block, one sub-tile");
+    gemm_w4_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  // Every ring slot holds one k-step.
+  const int SL = p.load_stages, SA = p.a_stages;  // SA: A slots per group
+  uint8_t* l_ring = smem;                         // SL x [activation box | raw chunk]
+  uint8_t* region = l_ring + SL * p.load_stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(region);
+  uint64_t* empty = full + SL;
+  uint64_t* afull = empty + SL;        // [2][SA] A slot written (one arrival per group step)
+  uint64_t* aempty = afull + 2 * SA;   // [2][SA] A slot consumed by its MMAs
+  uint64_t* drained = aempty + 2 * SA; // the MMA thread's final drain
+  const Ctl c = make_ctl(region, drained + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+  const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SL; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2 * SA; ++s) {
+      mbar_init(&afull[s], 1);
+      mbar_init(&aempty[s], 1);
+    }
+    mbar_init(drained, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&c.accf[b], 1);
+      mbar_init(&c.acce[b], kEpiThreads);
+    }
+    *c.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(c.tmem_slot, p.tmem_alloc);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *c.tmem_slot;
+  const Sched& sc = p.sc;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmap_x);
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      const uint32_t tx_bytes = static_cast<uint32_t>(kTileBytes) + b_bytes;
+      int i = 0;
+      Ring rl;
+      Seg g;
+      bool stop = false;
+      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
+        const int n_tile = g.tile % sc.n_tiles;
+        const int t_row = (g.tile / sc.n_tiles) * p.tok_tile;
+        const uint8_t* wsrc = p.wq + (static_cast<size_t>(n_tile) * p.kb_real + g.kb0) * kTileBytes;
+        for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL), wsrc += kTileBytes) {
+          const int s = rl.s;
+          if (!mbar_wait(&empty[s], rl.ph ^ 1u, p.wait_ns)) {
+            set_error(p.err, DEV_TIMEOUT_PRODUCER);
+            *c.abort_flag = 1;
+          }
+          if (*c.abort_flag) {
+            stop = true;
+            break;
+          }
+          uint8_t* st = l_ring + s * p.load_stage_bytes;
+          mbar_arrive_expect_tx(&full[s], tx_bytes);
+          bulk_load(st + b_bytes, wsrc, kTileBytes, &full[s], pol_w);
+          tma_load_2d(st, &tmap_x, &full[s], ks * 64, t_row, pol_x);
+        }
+      }
+      // Never leave the CTA with bulk copies still landing in its shared memory.
+      for (int j = max(0, i - SL); j < i; ++j)
+        mbar_wait(&full[j % SL], static_cast<uint32_t>(j / SL) & 1u, drain_ns(p.wait_ns));
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
+      const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(l_ring));
+      const uint32_t l_step = p.load_stage_bytes >> 4;
+      Ring rl, ra[2];
+      int i = 0;  // k-block index over all segments; group i & 1 dequantized it
+      Seg g;
+      bool stop = false;
+      for (int q = 0; get_seg(sc, cta, q, g); ++q) {
+        int buf;
+        uint32_t par;
+        acc_slot(q, buf, par);
+        if (!stop && !mbar_wait(&c.acce[buf], par ^ 1u, p.wait_ns)) {
+          set_error(p.err, DEV_TIMEOUT_MMA);
+          *c.abort_flag = 1;
+        }
+        if (*c.abort_flag) stop = true;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols;
+        for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, ++i, rl.next(SL)) {
+          const int grp = i & 1;
+          const int slot = grp * SA + ra[grp].s;
+          if (!mbar_wait(&afull[slot], ra[grp].ph, p.wait_ns)) {
+            set_error(p.err, DEV_TIMEOUT_MMA);
+            *c.abort_flag = 1;
+          }
+          if (*c.abort_flag) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_tmem = tmem_base + p.a_col0 + static_cast<uint32_t>(slot) * 32u;
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(rl.s * l_step);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (ks > g.kb0 || kk > 0) ? 1u : 0u);
+          mma_commit(&empty[rl.s]);
+          mma_commit(&aempty[slot]);
+          ra[grp].next(SA);
+        }
+        // Every segment ends with a commit, also after an abort, so the
+        // epilogue never waits on a barrier nobody signals.
+        mma_commit(&c.accf[buf]);
+      }
+      // all MMAs have completed before TMEM can be released
+      mma_commit(drained);
+      mbar_wait(drained, 0, drain_ns(p.wait_ns));
+    }
+  } else if (warp < kEpiWarp0) {
+    // ------------------------------------------------------------ dequantize
+    const int grp = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // TMEM lanes this warp may store to
+    const int row = quarter * 32 + lane;
+    const bool signaller = lane == 0 && warp == 2 + 4 * grp;
+    const uint32_t t_row = tmem_base + p.a_col0 + static_cast<uint32_t>(grp * SA) * 32u +
+                           (static_cast<uint32_t>(quarter * 32) << 16);
+    int i = 0;  // k-block index over all segments of this CTA (both groups)
+    Ring rl, ra;
+    bool stop = false;
+    Seg g;
+    for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
+      for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL)) {
+        if ((i & 1) != grp) continue;
+        const int s = rl.s;
+        const int a = ra.s;
+        bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
+        ok = ok && mbar_wait(&aempty[grp * SA + a], ra.ph ^ 1u, p.wait_ns);
+        if (!ok) {
+          set_error(p.err, DEV_TIMEOUT_CONSUMER);
+          *c.abort_flag = 1;
+        }
+        tc_fence_after();
+        // this thread's weight row of the k-block: 64 codes + (min, scale)
+        const uint8_t* raw = l_ring + s * p.load_stage_bytes + b_bytes;
+        const uint4 w0 = *reinterpret_cast<const uint4*>(raw + row * 32);
+        const uint4 w1 = *reinterpret_cast<const uint4*>(raw + row * 32 + 16);
+        const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
+        const __half2 m2 = __low2half2(mm);
+        const __half2 s2 = __high2half2(mm);
+        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t r[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 d = dequant8(words[j], s2, m2);
+          r[4 * j] = d.x;
+          r[4 * j + 1] = d.y;
+          r[4 * j + 2] = d.z;
+          r[4 * j + 3] = d.w;
+        }
+        __syncwarp();
+        tmem_st_x32(t_row + static_cast<uint32_t>(a) * 32u, r);
+        tmem_st_wait();
+        tc_fence_before();
+        // the whole group has stored its rows (or someone gave up)
+        if (bar_any<kGroupThreads>(2 + grp, !ok || *c.abort_flag)) {
+          stop = true;
+          break;
+        }
+        if (signaller) mbar_arrive(&afull[grp * SA + a]);
+        ra.next(SA);
+      }
+    }
+  } else {
+    epilogue_role(p, c, tmem_base, warp, lane);
+  }
+  teardown(p, c, tmem_base, warp);
+}
+
+// ---------------------------------------------------------------------------
+// general kernel: A tiles in shared memory, one MMA-issuing thread
+// ---------------------------------------------------------------------------
+// KS: 64-wide k-blocks per pipeline stage (k-step); two halve the mbarrier
+// hand-offs per tile, which bound decode-sized tiles.
+template <bool kW4, int KS>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const GemmParams p) {
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
   const int SL = p.load_stages, SA = p.a_stages;
-  constexpr uint32_t a_slot_bytes = KS * MT * kATileBytes;
-  uint8_t* a_ring = smem;                       // SA x [KS][MT] fp16 A tiles (4-bit weights only)
-  uint8_t* l_ring = smem + (kTS ? 0 : SA * a_slot_bytes);  // SL x load_stage_bytes
-  uint64_t* full = reinterpret_cast<uint64_t*>(l_ring + SL * p.load_stage_bytes);
+  constexpr uint32_t a_slot_bytes = KS * kATileBytes;
+  uint8_t* a_ring = smem;                       // SA x KS fp16 A tiles (4-bit weights only)
+  uint8_t* l_ring = smem + SA * a_slot_bytes;   // SL x load_stage_bytes
+  uint8_t* region = l_ring + SL * p.load_stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(region);
   uint64_t* empty = full + SL;
   uint64_t* afull = empty + SL;
   uint64_t* aempty = afull + SA;
-  uint64_t* accf = aempty + SA;  // [2]
-  uint64_t* acce = accf + 2;     // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* last_flag = abort_flag + 1;
-  volatile int* fin_count = abort_flag + 2;
-  int* fin_slots = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + kBarrierBytes / 2);  // [kMaxContrib]
-  float* epi_stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + kBarrierBytes);
+  uint64_t* drained = aempty + SA;
+  const Ctl c = make_ctl(region, drained + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
   const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;  // one 64-wide activation box
-  // load slot: 4-bit = [KS activation boxes | MT x KS raw chunks]; fp16 = [KS weight boxes | KS activation boxes]
+  // load slot: 4-bit = [KS activation boxes | KS raw chunks]; fp16 = [KS weight boxes | KS activation boxes]
   const uint32_t b_off = kW4 ? 0u : static_cast<uint32_t>(KS * kATileBytes);
   const uint32_t raw_off = KS * b_bytes;
-  constexpr int kTileCols = MT * 128;  // output features per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SL; ++s) {
@@ -328,21 +750,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&afull[s], kDequantThreads);
       mbar_init(&aempty[s], 1);
     }
+    mbar_init(drained, 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&accf[b], 1);
-      mbar_init(&acce[b], kEpiThreads);
+      mbar_init(&c.accf[b], 1);
+      mbar_init(&c.acce[b], kEpiThreads);
     }
-    *abort_flag = 0;
+    *c.abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, p.tmem_alloc);
+    tmem_alloc(c.tmem_slot, p.tmem_alloc);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_base = *c.tmem_slot;
   const Sched& sc = p.sc;
 
   if (warp == 0) {
@@ -352,6 +775,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!kW4) prefetch_tmap(&tmap_w);
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
+      const uint32_t tx_bytes =
+          KS * ((kW4 ? static_cast<uint32_t>(kTileBytes) : static_cast<uint32_t>(kATileBytes)) + b_bytes);
       int i = 0;
       Ring rl;
       Seg g;
@@ -359,28 +784,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
         const int n_tile = g.tile % sc.n_tiles;
         const int t_row = (g.tile / sc.n_tiles) * p.tok_tile;
-        const int mt_n = min(MT, p.n_sub - n_tile * MT);  // sub-tiles present in this tile
-        const uint32_t tx_bytes = kW4 ? KS * (static_cast<uint32_t>(mt_n * kTileBytes) + b_bytes)
-                                      : KS * (static_cast<uint32_t>(kATileBytes) + b_bytes);
-        const uint8_t* wsrc = p.wq + (static_cast<size_t>(n_tile) * MT * p.kb_real + g.kb0 * KS) * kTileBytes;
-        const size_t w_sub = static_cast<size_t>(p.kb_real) * kTileBytes;  // bytes per 128-row sub-tile
+        const uint8_t* wsrc = p.wq + (static_cast<size_t>(n_tile) * p.kb_real + g.kb0 * KS) * kTileBytes;
         for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL), wsrc += KS * kTileBytes) {
           const int s = rl.s;
           if (!mbar_wait(&empty[s], rl.ph ^ 1u, p.wait_ns)) {
             set_error(p.err, DEV_TIMEOUT_PRODUCER);
-            *abort_flag = 1;
+            *c.abort_flag = 1;
           }
-          if (*abort_flag) {
+          if (*c.abort_flag) {
             stop = true;
             break;
           }
           uint8_t* st = l_ring + s * p.load_stage_bytes;
           mbar_arrive_expect_tx(&full[s], tx_bytes);
-          if (kW4) {
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-              if (mt < mt_n) bulk_load(st + raw_off + mt * KS * kTileBytes, wsrc + mt * w_sub, KS * kTileBytes, &full[s], pol_w);
-          }
+          if (kW4) bulk_load(st + raw_off, wsrc, KS * kTileBytes, &full[s], pol_w);
 #pragma unroll
           for (int u = 0; u < KS; ++u) {
             const int kx = (ks * KS + u) * 64;
@@ -408,104 +825,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; get_seg(sc, cta, q, g); ++q) {
         int buf;
         uint32_t par;
-        acc_slot(p, q, buf, par);
-        if (!stop && !mbar_wait(&acce[buf], par ^ 1u, p.wait_ns)) {
+        acc_slot(q, buf, par);
+        if (!stop && !mbar_wait(&c.acce[buf], par ^ 1u, p.wait_ns)) {
           set_error(p.err, DEV_TIMEOUT_MMA);
-          *abort_flag = 1;
+          *c.abort_flag = 1;
         }
-        if (*abort_flag) stop = true;
+        if (*c.abort_flag) stop = true;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols;
-        const int mt_n = min(MT, p.n_sub - (g.tile % sc.n_tiles) * MT);
         for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, rl.next(SL), ra.next(SA)) {
           const int s = rl.s;
           const int sa = kW4 ? ra.s : 0;
           const bool ok = kW4 ? mbar_wait(&afull[sa], ra.ph, p.wait_ns) : mbar_wait(&full[s], rl.ph, p.wait_ns);
           if (!ok) {
             set_error(p.err, DEV_TIMEOUT_MMA);
-            *abort_flag = 1;
+            *c.abort_flag = 1;
           }
-          if (*abort_flag) {
+          if (*c.abort_flag) {
             stop = true;
             break;
           }
           const uint64_t adesc = adesc0 + static_cast<uint64_t>((kW4 ? sa : s) * a_step);
           const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * l_step);
-          if (kTS) {
-            tc_fence_after();
-            const uint32_t a_tmem = tmem_base + p.a_col0 + static_cast<uint32_t>(sa) * 32u;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (ks > g.kb0 || kk > 0) ? 1u : 0u);
-          } else
 #pragma unroll
           for (int u = 0; u < KS; ++u)
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-              if (mt < mt_n) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_f16_ss(d_tmem + mt * p.m_stride, adesc + (u * MT + mt) * (kATileBytes >> 4) + 2 * kk,
-                             bdesc + u * (b_bytes >> 4) + 2 * kk, idesc, (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
-              }
+            for (int kk = 0; kk < 4; ++kk)
+              mma_f16_ss(d_tmem, adesc + u * (kATileBytes >> 4) + 2 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk, idesc,
+                         (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[s]);
           if (kW4) mma_commit(&aempty[sa]);
         }
         // Every segment ends with a commit, also after an abort, so the
-        // epilogue and the teardown never wait on a barrier nobody signals.
-        mma_commit(&accf[buf]);
+        // epilogue never waits on a barrier nobody signals.
+        mma_commit(&c.accf[buf]);
       }
+      // all MMAs have completed before TMEM can be released
+      mma_commit(drained);
+      mbar_wait(drained, 0, drain_ns(p.wait_ns));
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ dequantize
-    if (kTS) {
-      // Warp w owns TMEM lanes 32*(w%4).. (the rows it may store to) and one
-      // 32-wide half of each k-block; each thread dequantizes one row's half.
-      const int quarter = warp & 3;
-      const int hf = (warp - 2) >> 2;
-      const int row = quarter * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + p.a_col0 + hf * 16;
-      Ring rl, ra;
-      Seg g;
-      bool stop = false;
-      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-        for (int ks = g.kb0; ks < g.kb1; ++ks, rl.next(SL), ra.next(SA)) {
-          const int s = rl.s;
-          const int sa = ra.s;
-          bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
-          ok = ok && mbar_wait(&aempty[sa], ra.ph ^ 1u, p.wait_ns);
-          if (!ok) {
-            set_error(p.err, DEV_TIMEOUT_CONSUMER);
-            *abort_flag = 1;
-          }
-          // tcgen05.st is warp-collective: the whole warp stops or none of it
-          if (__any_sync(0xffffffffu, !ok || *abort_flag != 0)) {
-            stop = true;
-            break;
-          }
-          tc_fence_after();
-          const uint8_t* raw = l_ring + s * p.load_stage_bytes + raw_off;
-          const uint4 c = *reinterpret_cast<const uint4*>(raw + row * 32 + hf * 16);
-          const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
-          const __half2 m2 = __low2half2(mm);
-          const __half2 s2 = __high2half2(mm);
-          const uint32_t words[4] = {c.x, c.y, c.z, c.w};
-          uint32_t r[16];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 d = dequant8(words[j], s2, m2);
-            r[4 * j] = d.x;
-            r[4 * j + 1] = d.y;
-            r[4 * j + 2] = d.z;
-            r[4 * j + 3] = d.w;
-          }
-          tmem_st_x16(t_row + static_cast<uint32_t>(sa) * 32u, r);
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&afull[sa]);
-        }
-      }
-    } else if (kW4) {
+    if (kW4) {
       const int ct = threadIdx.x - 64;
       const int row = ct >> 1;
       const int hf = ct & 1;
@@ -513,7 +874,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       Seg g;
       bool stop = false;
       for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-        const int mt_n = min(MT, p.n_sub - (g.tile % sc.n_tiles) * MT);
         for (int ks = g.kb0; ks < g.kb1; ++ks, rl.next(SL), ra.next(SA)) {
           const int s = rl.s;
           const int sa = ra.s;
@@ -521,191 +881,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = ok && mbar_wait(&aempty[sa], ra.ph ^ 1u, p.wait_ns);
           if (!ok) {
             set_error(p.err, DEV_TIMEOUT_CONSUMER);
-            *abort_flag = 1;
+            *c.abort_flag = 1;
           }
-          if (*abort_flag) {
+          if (*c.abort_flag) {
             stop = true;
             break;
           }
           const uint8_t* raw = l_ring + s * p.load_stage_bytes + raw_off;
-          uint4 c[MT][KS];
-          __half2 mm[MT][KS];
+          uint4 cw[KS];
+          __half2 mm[KS];
 #pragma unroll
-          for (int mt = 0; mt < MT; ++mt)
+          for (int u = 0; u < KS; ++u) {
+            cw[u] = *reinterpret_cast<const uint4*>(raw + u * kTileBytes + row * 32 + hf * 16);
+            mm[u] = *reinterpret_cast<const __half2*>(raw + u * kTileBytes + kTileCodeBytes + row * 4);
+          }
 #pragma unroll
-            for (int u = 0; u < KS; ++u) {
-              const uint8_t* chunk = raw + (mt * KS + u) * kTileBytes;
-              if (mt < mt_n) {
-                c[mt][u] = *reinterpret_cast<const uint4*>(chunk + row * 32 + hf * 16);
-                mm[mt][u] = *reinterpret_cast<const __half2*>(chunk + kTileCodeBytes + row * 4);
-              }
+          for (int u = 0; u < KS; ++u) {
+            const __half2 m2 = __low2half2(mm[u]);
+            const __half2 s2 = __high2half2(mm[u]);
+            uint8_t* arow = a_ring + sa * a_slot_bytes + u * kATileBytes + row * 128;
+            const uint32_t words[4] = {cw[u].x, cw[u].y, cw[u].z, cw[u].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int phys = (hf * 4 + j) ^ (row & 7);
+              *reinterpret_cast<uint4*>(arow + phys * 16) = dequant8(words[j], s2, m2);
             }
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int u = 0; u < KS; ++u) {
-              if (mt >= mt_n) continue;
-              const __half2 m2 = __low2half2(mm[mt][u]);
-              const __half2 s2 = __high2half2(mm[mt][u]);
-              uint8_t* arow = a_ring + sa * a_slot_bytes + (u * MT + mt) * kATileBytes + row * 128;
-              const uint32_t words[4] = {c[mt][u].x, c[mt][u].y, c[mt][u].z, c[mt][u].w};
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int phys = (hf * 4 + j) ^ (row & 7);
-                *reinterpret_cast<uint4*>(arow + phys * 16) = dequant8(words[j], s2, m2);
-              }
-            }
+          }
           fence_proxy_async_smem();
           mbar_arrive(&afull[sa]);
         }
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
-    const int et = threadIdx.x - kEpiWarp0 * 32;
-    const int qd = warp & 3;  // TMEM lane quarter this warp may access
-    Seg g;
-    for (int q = 0; get_seg(sc, cta, q, g); ++q) {
-      int buf;
-      uint32_t par;
-      acc_slot(p, q, buf, par);
-      const bool ok = mbar_wait(&accf[buf], par, drain_ns(p.wait_ns));
-      if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
-      tc_fence_after();
-      const bool aborted = epi_any(!ok || *abort_flag);
-      const int n_tile = g.tile % sc.n_tiles;
-      const int t_tile = g.tile / sc.n_tiles;
-      float* stg = epi_stage + (warp - kEpiWarp0) * 16 * 33;
-      const int tok0 = t_tile * p.tok_tile;
-      float* slot = g.full ? nullptr : p.partials + static_cast<size_t>(g.slot) * p.tok_tile * kTileCols;
-#pragma unroll 1
-      for (int mt = 0; mt < MT && !aborted; ++mt) {
-        const int frow = mt * 128 + qd * 32 + lane;  // feature row inside the tile
-        const uint32_t tbase = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + mt * p.m_stride +
-                               (static_cast<uint32_t>(qd * 32) << 16);
-        for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
-          uint32_t rr[16];
-          tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
-          tmem_ld_wait();
-          if (slot) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) slot[(c0 + j) * kTileCols + frow] = __uint_as_float(rr[j]);
-          } else {
-            // transpose 32 features x 16 tokens through shared memory so each
-            // lane finishes 16 consecutive features of one token
-#pragma unroll
-            for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = __uint_as_float(rr[j]);
-            __syncwarp();
-            const int jt = lane >> 1, hf = lane & 1;
-            const int tok = tok0 + c0 + jt;
-            const int f0 = n_tile * kTileCols + mt * 128 + qd * 32 + hf * 16;
-            if (tok < p.m && f0 < p.n) {
-              float v[16];
-#pragma unroll
-              for (int u = 0; u < 16; ++u) v[u] = stg[jt * 33 + hf * 16 + u];
-              store_row16(p, v, tok, f0);
-            }
-            __syncwarp();
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&acce[buf]);
-      if (slot == nullptr || aborted) continue;
-      // Partial tile: publish it, count it, and let the last contributor finish.
-      __threadfence();
-      epi_bar();
-      if (et == 0) {
-        int ns = 0;
-        if (sc.mode == SCHED_SPLITS) {
-          for (int part = 0; part < sc.splits && ns < kMaxContrib; ++part) fin_slots[ns++] = g.tile * sc.splits + part;
-        } else {
-          const long long t0 = static_cast<long long>(g.tile) * sc.kb_total;
-          for (int c = sk_first_contributor(sc, t0); c < sc.grid && sk_start(sc, c) < t0 + sc.kb_total &&
-                                                     ns < kMaxContrib;
-               ++c)
-            fin_slots[ns++] = 2 * c + (sk_start(sc, c) >= t0 ? 0 : 1);
-        }
-        *fin_count = ns;
-        const int old = atomicAdd(&p.counters[g.tile], 1);
-        *last_flag = old == ns - 1;
-      }
-      epi_bar();
-      const bool last = *last_flag;
-      const int ns = *fin_count;
-      if (last) {
-        __threadfence();
-        // Sum the slots in contributor order with coalesced 16-byte loads (two
-        // contributors in flight): thread et finishes 16 consecutive features
-        // of tokens et/8, et/8 + 16, ... for each 128-feature sub-tile.
-        const int tsub = et >> 3;
-        for (int mt = 0; mt < MT; ++mt) {
-          const int fg = mt * 128 + (et & 7) * 16;
-          const int f0 = n_tile * kTileCols + fg;
-          for (int c = tsub; c < p.tok_tile; c += 16) {
-            float acc[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) acc[u] = 0.f;
-            int k = 0;
-            for (; k + 1 < ns; k += 2) {
-              const float4* b0 = reinterpret_cast<const float4*>(
-                  p.partials + (static_cast<size_t>(fin_slots[k]) * p.tok_tile + c) * kTileCols + fg);
-              const float4* b1 = reinterpret_cast<const float4*>(
-                  p.partials + (static_cast<size_t>(fin_slots[k + 1]) * p.tok_tile + c) * kTileCols + fg);
-              float4 v0[4], v1[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                v0[u] = __ldcg(b0 + u);
-                v1[u] = __ldcg(b1 + u);
-              }
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                acc[4 * u] += v0[u].x + v1[u].x;
-                acc[4 * u + 1] += v0[u].y + v1[u].y;
-                acc[4 * u + 2] += v0[u].z + v1[u].z;
-                acc[4 * u + 3] += v0[u].w + v1[u].w;
-              }
-            }
-            if (k < ns) {
-              const float4* b0 = reinterpret_cast<const float4*>(
-                  p.partials + (static_cast<size_t>(fin_slots[k]) * p.tok_tile + c) * kTileCols + fg);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const float4 v = __ldcg(b0 + u);
-                acc[4 * u] += v.x;
-                acc[4 * u + 1] += v.y;
-                acc[4 * u + 2] += v.z;
-                acc[4 * u + 3] += v.w;
-              }
-            }
-            const int tok = tok0 + c;
-            if (tok < p.m && f0 < p.n) store_row16(p, acc, tok, f0);
-          }
-        }
-      }
-      epi_bar();  // everyone is done with the flag and the slot list before they are rewritten
-    }
+    epilogue_role(p, c, tmem_base, warp, lane);
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    // The last segment's accumulator commit completes only after every MMA of
-    // this CTA; wait for it so TMEM is never released under a running MMA.
-    if (lane == 0) {
-      Seg g;
-      int nq = 0;
-      while (get_seg(sc, cta, nq, g)) ++nq;
-      if (nq > 0) {
-        int buf;
-        uint32_t par;
-        acc_slot(p, nq - 1, buf, par);
-        mbar_wait(&accf[buf], par, drain_ns(p.wait_ns));
-      }
-    }
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_alloc);
-  }
+  teardown(p, c, tmem_base, warp);
 }
 
 // ---------------------------------------------------------------------------
@@ -745,15 +955,12 @@ bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, i
 
 struct Plan {
   int tok_tile, tok_tiles, n_tiles;
-  int ks;  // 64-wide k-blocks per pipeline stage
-  int mt;  // 128-row weight sub-tiles per output tile
-  bool ts;  // A (dequantized weights) in tensor memory
-  uint32_t a_col0;
+  bool decode;  // gemm_w4_decode_kernel
+  int ks;       // k-blocks per stage of gemm_tc_kernel
   Sched sc;
   int load_stages, a_stages;
   uint32_t load_stage_bytes;
-  uint32_t acc_cols, m_stride, tmem_alloc;
-  int nbuf;
+  uint32_t acc_cols, tmem_alloc, a_col0;
   size_t smem;
   size_t partial_bytes, counter_bytes;
 };
@@ -774,17 +981,15 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.tok_tiles = (m + 255) / 256;
     P.tok_tile = round_up((m + P.tok_tiles - 1) / P.tok_tiles, 16);
   }
-  // Decode-sized token tiles on 4-bit weights: two 128-row sub-tiles share
-  // each activation tile (half the L2 -> SM activation traffic per MMA), or,
-  // for a single sub-tile, two k-blocks per stage (half the hand-offs).
-  const bool decode_w4 = w_bits == 4 && P.tok_tile <= 160;
-  P.ts = false;  // measured slower than two k-blocks per shared-memory stage
-  P.mt = 1;
-  P.ks = decode_w4 && !P.ts && kb_real % 2 == 0 ? 2 : 1;
+  // Decode-sized tiles on 4-bit weights: two k-blocks per shared-memory stage
+  // (measured fastest on the OPT-30B decode shapes); the tensor-memory-A
+  // kernel takes the shapes with an odd number of k-blocks.
+  const bool dec = w_bits == 4 && P.tok_tile <= kDecodeMaxTok;
+  P.ks = dec && kb_real % 2 == 0 ? 2 : 1;
+  P.decode = dec && P.ks == 1;
   const int kb_total = kb_real / P.ks;  // k-steps per tile
-  const int min_iters = max(1, kMinItersPerCta / (P.ks * P.mt));
-  const int n_sub = (n + 127) / 128;
-  P.n_tiles = (n_sub + P.mt - 1) / P.mt;
+  const int min_iters = max(1, kMinItersPerCta / P.ks);
+  P.n_tiles = (n + 127) / 128;
   const int tiles = P.n_tiles * P.tok_tiles;
   const int sms = runtime().num_sms;
   Sched& s = P.sc;
@@ -794,7 +999,7 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   s.iters = static_cast<long long>(tiles) * kb_total;
   s.splits = 1;
   s.per = kb_total;
-  const size_t tile_bytes = static_cast<size_t>(P.tok_tile) * P.mt * 128 * sizeof(float);
+  const size_t tile_bytes = static_cast<size_t>(P.tok_tile) * 128 * sizeof(float);
   if (force_splits > 1) {
     s.mode = SCHED_SPLITS;
     s.per = (kb_total + force_splits - 1) / force_splits;
@@ -817,41 +1022,31 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
       s.grid = static_cast<int>(std::max<long long>(1, s.iters * (kMaxContrib - 2) / kb_total));
     P.partial_bytes = static_cast<size_t>(2) * s.grid * tile_bytes;
   }
-  if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * sizeof(int);
-  // TMEM: one accumulator set = mt sub-tiles x tok_tile fp32 columns; two sets
-  // when they fit in the 512 columns, so the epilogue overlaps the next segment.
-  P.m_stride = static_cast<uint32_t>(P.mt == 1 ? P.tok_tile : round_up(P.tok_tile, 32));
-  const uint32_t set = P.mt == 1 ? P.m_stride : P.mt * P.m_stride;
-  uint32_t set_pow2 = 32;
-  while (set_pow2 < set) set_pow2 <<= 1;
-  if (P.mt == 1) {
-    P.acc_cols = set_pow2;  // power-of-two sets
-    P.nbuf = 2;
-  } else {
-    P.acc_cols = set;
-    P.nbuf = 2 * set <= 512 ? 2 : 1;
-  }
-  if (P.ts) {
-    // two accumulator sets, then the A ring: 32 columns (128 x 64 fp16) per stage
-    P.acc_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
-    P.nbuf = 2;
-    P.a_col0 = 2 * P.acc_cols;
-  }
-  P.tmem_alloc = P.ts ? 512 : 32;
-  while (P.tmem_alloc < P.nbuf * P.acc_cols) P.tmem_alloc <<= 1;
+  if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * 2 * sizeof(int);
   const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
   const int b_bytes = P.tok_tile * 128;
   int a_slot = 0;
-  if (P.ts) {
-    P.a_stages = min(8, static_cast<int>((512 - P.a_col0) / 32));
-    P.load_stage_bytes = static_cast<uint32_t>(b_bytes + round_up(kTileBytes, 1024));
-  } else if (w_bits == 4) {
-    a_slot = P.ks * P.mt * kATileBytes;
-    P.a_stages = P.mt == 2 ? 3 : (P.ks == 2 ? 2 : (P.tok_tile > 128 && P.tok_tile != 144 ? 2 : 3));
-    P.load_stage_bytes = static_cast<uint32_t>(P.ks * b_bytes + round_up(P.mt * P.ks * kTileBytes, 1024));
+  if (P.decode) {
+    // TMEM: two accumulator buffers, then one A ring per group (32 columns =
+    // 128 rows x 64 fp16 per slot)
+    P.acc_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
+    P.a_col0 = 2 * P.acc_cols;
+    P.tmem_alloc = 512;
+    P.a_stages = min(4, static_cast<int>((512 - P.a_col0) / 64));
+    P.load_stage_bytes = static_cast<uint32_t>(b_bytes + kRawStageBytes);
   } else {
-    P.a_stages = 0;
-    P.load_stage_bytes = static_cast<uint32_t>(P.ks * (kATileBytes + b_bytes));
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
+    P.acc_cols = cols;
+    P.tmem_alloc = 2 * cols;
+    if (w_bits == 4) {
+      a_slot = P.ks * kATileBytes;
+      P.a_stages = P.ks == 2 ? 2 : (P.tok_tile > 128 && P.tok_tile != 144 ? 2 : 3);
+      P.load_stage_bytes = static_cast<uint32_t>(P.ks * b_bytes + round_up(P.ks * kTileBytes, 1024));
+    } else {
+      P.a_stages = 0;
+      P.load_stage_bytes = static_cast<uint32_t>(kATileBytes + b_bytes);
+    }
   }
   P.load_stages = min(kMaxLoadStages, (budget - P.a_stages * a_slot) / static_cast<int>(P.load_stage_bytes));
   P.smem = static_cast<size_t>(P.a_stages) * a_slot + static_cast<size_t>(P.load_stages) * P.load_stage_bytes +
@@ -859,22 +1054,31 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   return P;
 }
 
-template <bool kW4, int KS, int MT, bool kTS>
+// Raises the kernel's dynamic shared-memory limit once per process; one
+// instantiation (and so one flag) per kernel.
+template <auto kKernel>
 cudaError_t configure_once() {
   static cudaError_t status = cudaErrorNotReady;
   static std::once_flag once;
   std::call_once(once, [] {
-    status = cudaFuncSetAttribute(gemm_tc_kernel<kW4, KS, MT, kTS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+    status = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   });
   return status;
 }
 
-template <bool kW4, int KS, int MT, bool kTS = false>
-cudaError_t launch_variant(const Plan& P, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
+template <bool kW4, int KS>
+cudaError_t launch_general(const Plan& P, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                            cudaStream_t s) {
-  const cudaError_t e = configure_once<kW4, KS, MT, kTS>();
+  const cudaError_t e = configure_once<gemm_tc_kernel<kW4, KS>>();
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<kW4, KS, MT, kTS><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
+  gemm_tc_kernel<kW4, KS><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
+  return launched();
+}
+
+cudaError_t launch_decode(const Plan& P, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s) {
+  const cudaError_t e = configure_once<gemm_w4_decode_kernel>();
+  if (e != cudaSuccess) return e;
+  gemm_w4_decode_kernel<<<P.sc.grid, kThreads, P.smem, s>>>(tx, p);
   return launched();
 }
 
@@ -891,7 +1095,6 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   const Plan P = make_plan(a.m, a.n, a.k, a.w_bits, a.force_splits, a.force_tok_tile);
   const bool w4 = a.w_bits == 4;
   if (P.load_stages < 2) return cudaErrorInvalidValue;
-  cudaError_t e;
   CUtensorMap tx, tw;
   if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile)) return cudaErrorInvalidValue;
   if (w4) {
@@ -909,11 +1112,8 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.load_stages = P.load_stages;
   p.a_stages = P.a_stages;
   p.load_stage_bytes = P.load_stage_bytes;
-  p.n_sub = (a.n + 127) / 128;
   p.acc_cols = P.acc_cols;
-  p.m_stride = P.m_stride;
   p.tmem_alloc = P.tmem_alloc;
-  p.nbuf = P.nbuf;
   p.a_col0 = P.a_col0;
   p.sc = P.sc;
   p.bias = a.bias;
@@ -934,14 +1134,13 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
     if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
     p.partials = static_cast<float*>(ws);
     p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + align256(P.partial_bytes));
-    e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
+    const cudaError_t e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  if (w4 && P.ts) return launch_variant<true, 1, 1, true>(P, tx, tw, p, s);
-  if (w4 && P.mt == 2) return launch_variant<true, 1, 2>(P, tx, tw, p, s);
-  if (w4 && P.ks == 2) return launch_variant<true, 2, 1>(P, tx, tw, p, s);
-  if (w4) return launch_variant<true, 1, 1>(P, tx, tw, p, s);
-  return launch_variant<false, 1, 1>(P, tx, tw, p, s);
+  if (P.decode) return launch_decode(P, tx, p, s);
+  if (w4 && P.ks == 2) return launch_general<true, 2>(P, tx, tw, p, s);
+  if (w4) return launch_general<true, 1>(P, tx, tw, p, s);
+  return launch_general<false, 1>(P, tx, tw, p, s);
 }
 
 }  // namespace flexq
