@@ -199,6 +199,7 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const __half* __r
 // and a floating-point multiply-add.
 // ---------------------------------------------------------------------------
 constexpr int kStatN = 5;  // S, pm[2], wmax[2]
+constexpr int kUnroll = 4;  // independent 16-byte loads in flight per lane in the K and V passes
 
 __device__ __forceinline__ void block_reduce_stats(float (&v)[kStatN], float (*red)[kStatN]) {
 #pragma unroll
@@ -295,36 +296,50 @@ __global__ void __launch_bounds__(kThreads) attn_decode_q4_kernel(const __half* 
     }
   }
 
-  // pass 1: scores, 8 tokens per warp, 4 lanes per token
+  // pass 1: scores, 8 tokens per warp, 4 lanes per token.  kUnroll groups of
+  // tokens are loaded before any is used, so each warp keeps several 16-byte
+  // loads per lane in flight (the pass is bound by load latency otherwise).
   float mx = -INFINITY;
-  for (int base = warp * 8; base < len; base += kThreads / 4) {
-    const int t = base + (lane >> 2);
-    const bool valid = t < len;
-    float partial = 0.f;
-    if (valid) {
-      uint32_t cw[NW];
-      load_words<NW>(kw + static_cast<size_t>(t) * (D / 8) + c * NW, cw);
-      int dh = 0;
-      uint32_t dl = 0u;
+  constexpr int kStride = kThreads / 4;  // tokens per block-wide step
+  for (int base = warp * 8; base < len; base += kUnroll * kStride) {
+    uint32_t cw[kUnroll][NW];
+    __half2 msh[kUnroll];
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const uint32_t lo = cw[w] & 0x0F0F0F0Fu;
-        const uint32_t hi = (cw[w] >> 4) & 0x0F0F0F0Fu;
-        dh = __dp4a(static_cast<int>(lo), qh_e[w], dh);
-        dh = __dp4a(static_cast<int>(hi), qh_o[w], dh);
-        dl = __dp4a(lo, ql_e[w], dl);
-        dl = __dp4a(hi, ql_o[w], dl);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = base + u * kStride + (lane >> 2);
+      if (t < len) {
+        load_words<NW>(kw + static_cast<size_t>(t) * (D / 8) + c * NW, cw[u]);
+        msh[u] = km[static_cast<size_t>(t) * G + g];  // (min, scale)
       }
-      const float dot = (static_cast<float>(dh) * 256.0f + static_cast<float>(dl)) * inv_qscale;
-      const float2 ms = __half22float2(km[static_cast<size_t>(t) * G + g]);  // (min, scale)
-      partial = ms.y * dot + ms.x * qsum;
     }
-    partial += __shfl_xor_sync(0xffffffffu, partial, 1);
-    partial += __shfl_xor_sync(0xffffffffu, partial, 2);
-    if (valid) {
-      const float s = partial * inv_sqrt_d;
-      if (c == 0) sc[t] = s;
-      mx = fmaxf(mx, s);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = base + u * kStride + (lane >> 2);
+      const bool valid = t < len;
+      float partial = 0.f;
+      if (valid) {
+        int dh = 0;
+        uint32_t dl = 0u;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const uint32_t lo = cw[u][w] & 0x0F0F0F0Fu;
+          const uint32_t hi = (cw[u][w] >> 4) & 0x0F0F0F0Fu;
+          dh = __dp4a(static_cast<int>(lo), qh_e[w], dh);
+          dh = __dp4a(static_cast<int>(hi), qh_o[w], dh);
+          dl = __dp4a(lo, ql_e[w], dl);
+          dl = __dp4a(hi, ql_o[w], dl);
+        }
+        const float dot = (static_cast<float>(dh) * 256.0f + static_cast<float>(dl)) * inv_qscale;
+        const float2 ms = __half22float2(msh[u]);
+        partial = ms.y * dot + ms.x * qsum;
+      }
+      partial += __shfl_xor_sync(0xffffffffu, partial, 1);
+      partial += __shfl_xor_sync(0xffffffffu, partial, 2);
+      if (valid) {
+        const float s = partial * inv_sqrt_d;
+        if (c == 0) sc[t] = s;
+        mx = fmaxf(mx, s);
+      }
     }
   }
   const float M = block_reduce(mx, &red[0][0], true);
@@ -377,18 +392,28 @@ __global__ void __launch_bounds__(kThreads) attn_decode_q4_kernel(const __half* 
   uint32_t ah[DPV], al[DPV];
 #pragma unroll
   for (int e = 0; e < DPV; ++e) ah[e] = al[e] = 0u;
-  for (int blk = warp; blk < nblk; blk += kThreads / 32) {
-    uint32_t vwd[DPV];
-    load_words<DPV>(vw + static_cast<size_t>(blk) * D + lane * DPV, vwd);
-    const uint4 wp = wpk[blk * G + gv];
+  constexpr int kWarps = kThreads / 32;
+  for (int blk0 = warp; blk0 < nblk; blk0 += kUnroll * kWarps) {
+    uint32_t vwd[kUnroll][DPV];
 #pragma unroll
-    for (int e = 0; e < DPV; ++e) {
-      const uint32_t lo = vwd[e] & 0x0F0F0F0Fu;
-      const uint32_t hi = (vwd[e] >> 4) & 0x0F0F0F0Fu;
-      al[e] = __dp4a(lo, wp.x, al[e]);
-      al[e] = __dp4a(hi, wp.y, al[e]);
-      ah[e] = __dp4a(lo, wp.z, ah[e]);
-      ah[e] = __dp4a(hi, wp.w, ah[e]);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int blk = blk0 + u * kWarps;
+      if (blk < nblk) load_words<DPV>(vw + static_cast<size_t>(blk) * D + lane * DPV, vwd[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int blk = blk0 + u * kWarps;
+      if (blk >= nblk) break;
+      const uint4 wp = wpk[blk * G + gv];
+#pragma unroll
+      for (int e = 0; e < DPV; ++e) {
+        const uint32_t lo = vwd[u][e] & 0x0F0F0F0Fu;
+        const uint32_t hi = (vwd[u][e] >> 4) & 0x0F0F0F0Fu;
+        al[e] = __dp4a(lo, wp.x, al[e]);
+        al[e] = __dp4a(hi, wp.y, al[e]);
+        ah[e] = __dp4a(lo, wp.z, ah[e]);
+        ah[e] = __dp4a(hi, wp.w, ah[e]);
+      }
     }
   }
 #pragma unroll
