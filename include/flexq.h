@@ -132,11 +132,13 @@ flexq_status flexq_quantize_weight_q4(const void* w_dev, int n_out, int k_in, vo
  * flags: 1 = + bias[n], 2 = GELU (erf form) after the bias, 4 = + residual
  * [m][ld_res] last, 8 = write fp32 (alone).  y_dev fp16 (or fp32) [m][ldy].
  * ws: fp32 partial output tiles when K is shared out across CTAs (small
- * grids) plus one counter per tile; size from flexq_linear_workspace with the
- * same force_splits (0 means none needed).  force_splits = 0 lets the library
- * choose (whole tiles per SM when there are many, equal shares of all
- * k-blocks per SM when there are few); s > 1 cuts every tile's K into s parts
- * (tests); 1 forbids splitting K. */
+ * grids) plus two counters per tile (contributors arrived, partials
+ * published; zeroed on the stream by the call); size from
+ * flexq_linear_workspace with the same force_splits (0 means none needed).
+ * force_splits = 0 lets the library choose (whole tiles per SM when there are
+ * many, equal shares of all k-blocks per SM when there are few); s > 1 cuts
+ * every tile's K into s parts (tests); 1 forbids splitting K.  A split tile is
+ * summed in a fixed contributor order, so results do not depend on timing. */
 size_t flexq_linear_workspace(int m, int n, int k, int w_bits, int force_splits);
 flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_bits, int m, int n,
                           int k, const void* bias_dev, const void* residual_dev, int ld_res,
@@ -331,7 +333,7 @@ typedef enum {
  * launch is bracketed by two CUDA events on its stream (adds a little time;
  * one host thread at a time).  stop synchronises `stream` and writes, per
  * kind, the summed device milliseconds and the number of bracketed calls
- * (a linear layer's call may hold a K-split finishing kernel as well). */
+ * (a linear layer's call also holds the memset of its split-tile counters). */
 flexq_status flexq_profile_start(void);
 flexq_status flexq_profile_stop(void* stream, float* total_ms /* [FLEXQ_K_COUNT] */,
                                 int* calls /* [FLEXQ_K_COUNT] */);
