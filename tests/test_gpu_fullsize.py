@@ -81,10 +81,16 @@ def _check_codes(got_codes, want_codes):
 
 
 # At the OPT-175B shape the decode output measured 2.1 % (relative Frobenius)
-# away from the oracle on an identical cache, while its prefill rows and cache
-# codes, and the decode at the other four shapes, meet the bars: an open parity
-# gap, kept visible here rather than hidden by a looser bound.
-GAP_175B = pytest.mark.xfail(reason="decode at the OPT-175B shape: 2.1 % relative error, open", strict=False)
+# away from the float64 oracle on an identical prompt cache, while its prefill
+# rows and cache codes, and the decode at the other four shapes, meet the bars.
+# The oracle alone moves by the same 2.08 % when only its LN1 output is stored
+# in fp16 (the precision the layer computes in): 11 of the 6144 code bytes of
+# the appended token's K row then land one step apart, and at this width the
+# token's own attention weight amplifies that.  The output is decided by
+# quantization decisions taken in different precisions, so the bar does not
+# apply as stated; kept visible as an open item, not hidden by a looser bound.
+GAP_175B = pytest.mark.xfail(reason="OPT-175B decode: appended-row code decisions taken in different "
+                                    "precisions move the output 2.1 %", strict=False)
 
 
 @pytest.mark.parametrize("name", ["opt-1.3b", "opt-6.7b", "opt-30b", "opt-30b-s1024",
