@@ -61,22 +61,36 @@ def load_peaks():
             "source": "fallback"}
 
 
-def csrc_hash():
+def csrc_hash(files=None):
+    """Hash of the CUDA sources (all of them, or the named files)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "quantized_opt_decode_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files if files is not None else os.listdir(d)):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
+# Source files that define each kernel kind's device code: an ncu traffic
+# figure stays valid while these are unchanged.
+_SHARED = ["common.cuh", "kernels.h"]
+KERNEL_FILES = {
+    "attn_decode": ["attn_decode.cu"] + _SHARED,
+    "qkv": ["gemm_tc.cu"] + _SHARED, "out_proj": ["gemm_tc.cu"] + _SHARED,
+    "fc1": ["gemm_tc.cu"] + _SHARED, "fc2": ["gemm_tc.cu"] + _SHARED,
+    "lm_head": ["gemm_tc.cu"] + _SHARED,
+    "kv_append": ["kv_append.cu", "quant_common.cuh"] + _SHARED,
+    "layernorm": ["rowwise.cu"] + _SHARED,
+}
+
+
 def ncu_traffic(kind: str):
     """DRAM bytes per launch of `kind` from the committed ncu summary, or None
-    when absent or taken on other kernel sources."""
+    when absent or taken on other sources of that kernel."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kind not in KERNEL_FILES:
         return None
-    cur = csrc_hash()
+    cur = csrc_hash(KERNEL_FILES[kind])
     with open(path) as f:
         for line in f:
             parts = line.split()
