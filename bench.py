@@ -99,6 +99,23 @@ def ncu_traffic(kind: str):
     return None
 
 
+def max_over_ranks(x: float, device: str = "cuda") -> float:
+    """The largest x over all ranks (all ranks must call it, in the same
+    order); x itself when there is no process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def prompt_tensor_id(rank: int) -> int:
+    """Each replica generates its own block of prompts."""
+    return synth.TID_PROMPT + 7919 * rank
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle samples every 200 ms while active."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -323,7 +340,7 @@ def run_flexq(args, p):
     with torch.cuda.stream(stream):
         dm = DeviceModel(p, b=b, max_len=s + n, stream=stream)
         prompts = torch.empty(b, s, dtype=torch.int32, device="cuda")
-        fq.flexq_synth_tokens(prompts, b * s, synth.config_seed(p), synth.TID_PROMPT + 7919 * rank,
+        fq.flexq_synth_tokens(prompts, b * s, synth.config_seed(p), prompt_tensor_id(rank),
                               p["vocab"], stream=stream)
         out = torch.zeros(b, n, dtype=torch.int32, device="cuda")
         ws_n = fq.flexq_generate_workspace(dm.struct, b, s, gbs)
@@ -368,11 +385,7 @@ def run_flexq(args, p):
         if world > 1:
             dist.barrier()
     clocks = clk.summary()
-    ms = t0.elapsed_time(t1) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps)
     fq.flexq_device_status(stream)
     value = world * b * (n - 1) / (ms / 1e3)
 
@@ -421,11 +434,7 @@ def run_flexq(args, p):
                 e2e_step()
             a1.record(stream)
         stream.synchronize()
-        e_ms = a0.elapsed_time(a1) / args.e2e_steps
-        if world > 1:
-            tt = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps)
         e2e = {"value": round(world * b * n / (e_ms / 1e3), 2), "unit": "tokens/s",
                "h2d_bytes_per_step": b * s * 4, "d2h_bytes_per_step": b * n * 4,
                "ms_per_step": round(e_ms, 2),
