@@ -126,3 +126,24 @@ def test_generate_rejects_indivisible_gpu_batch(fq):
     st = fq._lib.flexq_generate(C.byref(m), 0x5000, 4, 32, 10, 4, 0x6000, 0x7000, 1 << 30, None,
                                 None)
     assert st == 1 and "max_pos" in fq.flexq_last_error()
+
+
+def test_package_builds_from_scratch_and_binding_fails_loudly(tmp_path):
+    """Without libflexq.so the package still imports (so its build module can
+    compile the library on a fresh checkout), and the binding refuses to load:
+    there is no fallback path."""
+    import shutil
+    import subprocess
+    import sys
+    src = os.path.join(ROOT, "quantized_opt_decode_b200")
+    dst = tmp_path / "quantized_opt_decode_b200"
+    dst.mkdir()
+    for f in os.listdir(src):
+        if f.endswith(".py"):
+            shutil.copy(os.path.join(src, f), dst / f)
+    code = ("import quantized_opt_decode_b200 as q, quantized_opt_decode_b200.build as b\n"
+            "try:\n    q.flexq\nexcept ImportError as e:\n    print('refused:', e)\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True,
+                       env=dict(os.environ, PYTHONPATH=str(tmp_path)))
+    assert r.returncode == 0, r.stderr
+    assert "refused:" in r.stdout and "libflexq.so" in r.stdout
