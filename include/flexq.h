@@ -222,7 +222,11 @@ flexq_status flexq_kv_append(const flexq_config* cfg, const flexq_kv* kv, const 
 
 /* Decode attention: out[i][j*d ..] = softmax(q_ij K_ij^T / sqrt(d)) V_ij over
  * slots 0..len-1 of the cache (dequantized in 4-bit mode).  q_dev fp16
- * [b][ldq] (head j at columns j*d), out_dev fp16 [b][ldo]. */
+ * [b][ldq] (head j at columns j*d), out_dev fp16 [b][ldo].  In 4-bit mode the
+ * dequantization is folded into the sums (scale * sum q*code + min * sum q),
+ * which are formed with integer dot products: q as 15-bit fixed point per
+ * head row and the softmax weights as 16-bit fixed point per 8-token block
+ * and group (relative error well below fp16 output rounding). */
 flexq_status flexq_attention_decode(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev,
                                     int ldq, int b, int len, void* out_dev, int ldo, void* stream);
 
