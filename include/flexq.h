@@ -226,7 +226,7 @@ flexq_status flexq_kv_append(const flexq_config* cfg, const flexq_kv* kv, const 
  * dequantization is folded into the sums (scale * sum q*code + min * sum q),
  * which are formed with integer dot products: q as 15-bit fixed point per
  * head row and the softmax weights as 16-bit fixed point per 8-token block
- * and group (relative error well below fp16 output rounding). */
+ * and group (held to the layer tolerance by the parity tests). */
 flexq_status flexq_attention_decode(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev,
                                     int ldq, int b, int len, void* out_dev, int ldo, void* stream);
 
