@@ -191,6 +191,8 @@ def kernel_work(p: dict, kind: str, M: int, L_avg: float):
         return byts, 2.0 * M * n * k
     if kind == "attn_decode":
         return M * a * L_avg * 2 * kvb + 2 * M * h * 2, 4.0 * M * L_avg * h
+    if kind == "attn_prefill":  # causal: half of the s x s score and value products
+        return M * h * 2 * 4, 2.0 * M * L_avg * h
     if kind == "kv_append":
         return M * 2 * h * 2 + M * a * 2 * kvb, 0.0
     if kind == "layernorm":
@@ -202,6 +204,39 @@ def kernel_work(p: dict, kind: str, M: int, L_avg: float):
     if kind == "embed":
         return M * h * 6, 0.0
     return 0.0, 0.0
+
+
+def roof_time(p, kind, M, L, peaks) -> float:
+    """Seconds one call of `kind` takes at its roofline: the larger of its
+    algorithmic bytes at the measured HBM copy rate and its flops at the
+    measured sustained dense rate."""
+    byts, flops = kernel_work(p, kind, M, L)
+    return max(byts / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops_sustained"] * 1e12))
+
+
+def step_ceilings(p: dict, gbs: int, peaks: dict) -> dict:
+    """Tokens/s the decode phase and the prefill column would reach if every
+    kernel they launch ran at its own roofline (the per-kernel rooflines
+    summed over the launches of the step, in the launch order of
+    flexq_generate: per column and GPU batch the embedding, l layer steps,
+    the final LayerNorm, the tied LM head and the greedy choice)."""
+    b, s, n, layers = p["b"], p["s"], p["n"], p["layers"]
+    batches = b // gbs
+
+    def column(M_rows, M_head, L, attn):
+        t = roof_time(p, "embed", M_rows, L, peaks)
+        layer = (2 * roof_time(p, "layernorm", M_rows, L, peaks) + roof_time(p, "qkv", M_rows, L, peaks)
+                 + roof_time(p, "kv_append", M_rows, L, peaks) + roof_time(p, attn, M_rows, L, peaks)
+                 + roof_time(p, "out_proj", M_rows, L, peaks) + roof_time(p, "fc1", M_rows, L, peaks)
+                 + roof_time(p, "fc2", M_rows, L, peaks))
+        t += layers * layer
+        t += (roof_time(p, "layernorm", M_head, L, peaks) + roof_time(p, "lm_head", M_head, L, peaks)
+              + roof_time(p, "argmax", M_head, L, peaks))
+        return t
+
+    t_dec = sum(batches * column(gbs, gbs, s + j + 1, "attn_decode") for j in range(1, n))
+    t_pre = batches * column(gbs * s, gbs, s, "attn_prefill")
+    return {"decode_tokens_per_s": b * (n - 1) / t_dec, "prefill_tokens_per_s": b * s / t_pre}
 
 
 def roofline(p, kind, calls, ms_total, M, L_avg, peaks):
@@ -411,6 +446,7 @@ def run_flexq(args, p):
     rl = roofline(p, dom, prof[dom][1], prof[dom][0], gbs, L_avg, peaks)
     rl["traffic"] = ncu_traffic(dom)
     rl.pop("algorithmic_per_launch", None)
+    ceil = step_ceilings(p, gbs, peaks)
 
     # end to end through flexq_generate: prompts from pinned host memory,
     # tokens back to pinned host memory, all inside the timed region
@@ -462,7 +498,15 @@ def run_flexq(args, p):
             "roofline": rl,
             "kernels": kernels,
             "prefill": {"ms": round(prefill_ms, 2),
-                        "tokens_per_s": round(world * b * s / (prefill_ms / 1e3), 1)},
+                        "tokens_per_s": round(world * b * s / (prefill_ms / 1e3), 1),
+                        "frac_of_ceiling": round(world * b * s / (prefill_ms / 1e3)
+                                                 / (world * ceil["prefill_tokens_per_s"]), 4)},
+            "ceiling": {"decode_tokens_per_s": round(world * ceil["decode_tokens_per_s"], 1),
+                        "decode_frac": round(value / (world * ceil["decode_tokens_per_s"]), 4),
+                        "prefill_tokens_per_s": round(world * ceil["prefill_tokens_per_s"], 1),
+                        "what": "every launched kernel at its own roofline (algorithmic bytes at the "
+                                "measured HBM copy rate or flops at the measured sustained dense rate, "
+                                "whichever is slower), summed over the step"},
             "gpu_launches": int(launches),
             "gpu_launches_per_step": int(launches // max(1, args.steps)),
             "clocks": clocks,

@@ -1,0 +1,46 @@
+"""The benchmark's step ceiling (every launched kernel at its own roofline,
+summed over the step) against the closed form of the per-layer decode
+ceiling: GEMMs max(12 h^2 B_w / BW, 24 b h^2 / P), attention b L 2h B_kv / BW,
+plus the tied LM head max(2 V h / BW, 2 b V h / P) per column."""
+import importlib.util
+import os
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+bench = importlib.util.module_from_spec(spec)
+spec.loader.exec_module(bench)
+
+PEAKS = {"hbm_gbs": 6545.3, "bf16_tflops": 1661.0, "bf16_tflops_sustained": 1397.6, "source": "test"}
+
+
+def _closed_form(p):
+    BW, P = PEAKS["hbm_gbs"] * 1e9, PEAKS["bf16_tflops_sustained"] * 1e12
+    b, s, n, l, h, V = p["gpu_batch"], p["s"], p["n"], p["layers"], p["h"], p["vocab"]
+    bw = 0.5625 if p["w_bits"] == 4 else 2.0
+    bkv = 0.5625 if p["kv_bits"] == 4 else 2.0
+    t = 0.0
+    for j in range(1, n):
+        L = s + j + 1
+        layer = max(12 * h * h * bw / BW, 24 * b * h * h / P) + b * L * 2 * h * bkv / BW
+        t += l * layer + max(2 * V * h / BW, 2 * b * V * h / P)
+    return p["gpu_batch"] * (n - 1) / t
+
+
+def test_decode_ceiling_matches_closed_form():
+    for name in ("opt-1.3b", "opt-30b", "opt-30b-s1024", "opt-175b"):
+        p = dict(synth.CONFIGS[name])
+        got = bench.step_ceilings(p, p["gpu_batch"], PEAKS)["decode_tokens_per_s"]
+        want = _closed_form(p)
+        # the closed form leaves out activations, LayerNorm, the append and the argmax
+        assert 0.93 * want < got <= want, (name, got, want)
+
+
+def test_prefill_ceiling_is_tensor_bound_at_30b():
+    p = dict(synth.CONFIGS["opt-30b"])
+    b, s, h, l = p["b"], p["s"], p["h"], p["layers"]
+    flops = l * (24 * b * s * h * h + 2 * b * s * s * h)
+    want = b * s / (flops / (PEAKS["bf16_tflops_sustained"] * 1e12))
+    got = bench.step_ceilings(p, p["gpu_batch"], PEAKS)["prefill_tokens_per_s"]
+    assert 0.95 * want < got <= want, (got, want)
