@@ -48,7 +48,7 @@ typedef enum {
   FLEXQ_ERR_CUDA = 2,        /* a CUDA call or kernel launch failed */
   FLEXQ_ERR_WORKSPACE = 3,   /* workspace pointer null or too small */
   FLEXQ_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up */
-  FLEXQ_ERR_UNSUPPORTED = 5, /* valid request this build does not handle */
+  FLEXQ_ERR_UNSUPPORTED = 5, /* valid request the library does not handle */
   FLEXQ_ERR_DEVICE = 6       /* a kernel reported a bad device-side input */
 } flexq_status;
 

@@ -317,7 +317,7 @@ def generate(m: Model, prompts: np.ndarray, n: int, forced: np.ndarray | None = 
     Prefill over the prompt yields token 1; each of the n-1 decode steps feeds
     the previous token at position s + j - 1 and yields the next one.  With
     ``forced`` [b, n] the next input is forced[:, j-1] instead of the oracle's
-    own choice (teacher forcing, used to judge another generator's choices)."""
+    own choice (teacher forcing, used to check another generator's choices)."""
     cfg = m.cfg
     b, s = prompts.shape
     caches = [KVCache(cfg, b, s + n, cfg.kv_bits) for _ in range(cfg.layers)]
