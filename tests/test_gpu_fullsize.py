@@ -108,7 +108,7 @@ def _check_codes(got_codes, want_codes):
 # the appended token's K row then land one step apart, and at this width the
 # token's own attention weight amplifies that.  So at this shape the decode
 # reference takes the appended row's code decisions from an fp16 LN1 output
-# (the task's rule: both sides decide in the same precision).  That comparison
+# (a quantization decision is taken in the same precision on both sides).  That comparison
 # has not run on a GPU yet, so the case stays marked until it has.
 DECIDE_IN_F16 = {"opt-175b"}
 GAP_175B = pytest.mark.xfail(reason="OPT-175B decode against the fp16-LN1 reference: not yet confirmed "
