@@ -982,8 +982,10 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.tok_tile = round_up((m + P.tok_tiles - 1) / P.tok_tiles, 16);
   }
   // Decode-sized tiles on 4-bit weights: two k-blocks per shared-memory stage
-  // (measured fastest on the OPT-30B decode shapes); the tensor-memory-A
-  // kernel takes the shapes with an odd number of k-blocks.
+  // (measured fastest on the OPT-30B decode shapes).  Where K has an odd
+  // number of k-blocks two per stage do not divide it, and the tensor-memory-A
+  // kernel takes the shape (its speed against one k-block per stage in the
+  // shared-memory kernel is unmeasured; every benchmark shape has even K/64).
   const bool dec = w_bits == 4 && P.tok_tile <= kDecodeMaxTok;
   P.ks = dec && kb_real % 2 == 0 ? 2 : 1;
   P.decode = dec && P.ks == 1;
