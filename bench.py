@@ -223,19 +223,25 @@ def step_ceilings(p: dict, gbs: int, peaks: dict) -> dict:
     b, s, n, layers = p["b"], p["s"], p["n"], p["layers"]
     batches = b // gbs
 
-    def column(M_rows, M_head, L, attn):
-        t = roof_time(p, "embed", M_rows, L, peaks)
-        layer = (2 * roof_time(p, "layernorm", M_rows, L, peaks) + roof_time(p, "qkv", M_rows, L, peaks)
-                 + roof_time(p, "kv_append", M_rows, L, peaks) + roof_time(p, attn, M_rows, L, peaks)
-                 + roof_time(p, "out_proj", M_rows, L, peaks) + roof_time(p, "fc1", M_rows, L, peaks)
-                 + roof_time(p, "fc2", M_rows, L, peaks))
-        t += layers * layer
-        t += (roof_time(p, "layernorm", M_head, L, peaks) + roof_time(p, "lm_head", M_head, L, peaks)
-              + roof_time(p, "argmax", M_head, L, peaks))
+    def column(rows_per_batch, embed_rows, L, attn):
+        # embedding over the whole block, then every layer for every GPU
+        # batch, then the final LayerNorm, LM head and greedy choice over the
+        # block's last rows
+        t = roof_time(p, "embed", embed_rows, L, peaks)
+        layer = (2 * roof_time(p, "layernorm", rows_per_batch, L, peaks)
+                 + roof_time(p, "qkv", rows_per_batch, L, peaks)
+                 + roof_time(p, "kv_append", rows_per_batch, L, peaks)
+                 + roof_time(p, attn, rows_per_batch, L, peaks)
+                 + roof_time(p, "out_proj", rows_per_batch, L, peaks)
+                 + roof_time(p, "fc1", rows_per_batch, L, peaks)
+                 + roof_time(p, "fc2", rows_per_batch, L, peaks))
+        t += layers * batches * layer
+        t += (roof_time(p, "layernorm", b, L, peaks) + roof_time(p, "lm_head", b, L, peaks)
+              + roof_time(p, "argmax", b, L, peaks))
         return t
 
-    t_dec = sum(batches * column(gbs, gbs, s + j + 1, "attn_decode") for j in range(1, n))
-    t_pre = batches * column(gbs * s, gbs, s, "attn_prefill")
+    t_dec = sum(column(gbs, b, s + j + 1, "attn_decode") for j in range(1, n))
+    t_pre = column(gbs * s, b * s, s, "attn_prefill")
     return {"decode_tokens_per_s": b * (n - 1) / t_dec, "prefill_tokens_per_s": b * s / t_pre}
 
 
@@ -435,10 +441,12 @@ def run_flexq(args, p):
     for kind, (kms, calls) in prof.items():
         if calls == 0:
             continue
-        M = b if kind not in ("lm_head", "argmax", "embed") else b
-        rl = roofline(p, kind, calls, kms, gbs if kind in ("qkv", "out_proj", "fc1", "fc2",
-                                                            "attn_decode", "kv_append",
-                                                            "layernorm") else M, L_avg, peaks)
+        # rows per call: one GPU batch inside the layer steps, the whole block
+        # for the embedding, LM head and argmax (the final LayerNorm's b rows
+        # are counted at the GPU-batch size, which equals b in the default run)
+        M = gbs if kind in ("qkv", "out_proj", "fc1", "fc2", "attn_decode", "kv_append",
+                            "layernorm") else b
+        rl = roofline(p, kind, calls, kms, M, L_avg, peaks)
         kernels[kind] = {"calls": calls, "ms": round(kms, 3), "share": round(kms / total, 4),
                          "avg_us": round(kms / calls * 1e3, 2), "bound": rl["bound"],
                          "achieved": rl["achieved"], "unit": rl["unit"], "frac": rl["frac"]}
