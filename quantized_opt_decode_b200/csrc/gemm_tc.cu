@@ -1097,6 +1097,11 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   const Plan P = make_plan(a.m, a.n, a.k, a.w_bits, a.force_splits, a.force_tok_tile);
   const bool w4 = a.w_bits == 4;
   if (P.load_stages < 2) return cudaErrorInvalidValue;
+  // mbarriers the kernel lays out before its control words (make_ctl):
+  // decode: full/empty per load stage, afull/aempty per A slot of each group,
+  // the drain barrier, accf/acce x 2; general: the same with one A ring
+  const int n_bars = P.decode ? 2 * P.load_stages + 4 * P.a_stages + 5 : 2 * P.load_stages + 2 * P.a_stages + 5;
+  if (n_bars > kMaxBarriers) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
   if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile)) return cudaErrorInvalidValue;
   if (w4) {
