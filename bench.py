@@ -245,22 +245,99 @@ def step_ceilings(p: dict, gbs: int, peaks: dict) -> dict:
     return {"decode_tokens_per_s": b * (n - 1) / t_dec, "prefill_tokens_per_s": b * s / t_pre}
 
 
-def roofline(p, kind, calls, ms_total, M, L_avg, peaks):
-    byts, flops = kernel_work(p, kind, M, L_avg)
-    t = ms_total / calls / 1e3
+def phase_work(p: dict, kind: str, calls: int, gbs: int, phase: str, columns: int):
+    """(bytes, flops) of all `calls` launches of `kind` in one profiled pass of
+    a phase ("decode": the n-1 decode columns; "prefill": the prefill column).
+    Inside the layer steps a call covers one GPU batch (gbs rows, or gbs * s
+    in the prefill); the embedding, the final LayerNorm, the LM head and the
+    argmax cover the whole block once per column (the final LayerNorm shares
+    its kind with the layer LayerNorms: `columns` of the calls are final)."""
+    b, s, n = p["b"], p["s"], p["n"]
+    rows = gbs * s if phase == "prefill" else gbs
+    L = s if phase == "prefill" else s + n / 2.0
+    if kind in ("lm_head", "argmax"):
+        byts, flops = kernel_work(p, kind, b, L)
+        return calls * byts, calls * flops
+    if kind == "embed":
+        byts, flops = kernel_work(p, kind, b * s if phase == "prefill" else b, L)
+        return calls * byts, calls * flops
+    if kind == "layernorm":
+        n_final = min(columns, calls)
+        bl, _ = kernel_work(p, kind, rows, L)
+        bf, _ = kernel_work(p, kind, b, L)
+        return (calls - n_final) * bl + n_final * bf, 0.0
+    byts, flops = kernel_work(p, kind, rows, L)
+    return calls * byts, calls * flops
+
+
+def roofline(kind, byts, flops, seconds, peaks):
+    """Achieved rate of `kind` (all its launches in a profiled pass) against
+    its roof: the tensor pipe when its arithmetic intensity is above the
+    ridge of the measured peaks, HBM otherwise."""
     ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     if flops > 0 and flops / max(byts, 1.0) > ridge:
-        ach = flops / t / 1e12
+        ach = flops / seconds / 1e12
         peak = peaks["bf16_tflops_sustained"]
         return {"kernel": kind, "bound": "tensor", "achieved": round(ach, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-                "peak_note": f"{peaks['source']} dense bf16 sustained (fp16 nominal ratio 1:1)",
-                "algorithmic_per_launch": {"flops": flops, "bytes": byts}}
-    ach = byts / t / 1e9
+                "peak_note": f"{peaks['source']} dense bf16 sustained (fp16 nominal ratio 1:1)"}
+    ach = byts / seconds / 1e9
     peak = peaks["hbm_gbs"]
     return {"kernel": kind, "bound": "hbm", "achieved": round(ach, 1), "peak": peak,
-            "unit": "GB/s", "frac": round(ach / peak, 4), "peak_note": f"{peaks['source']} HBM copy",
-            "algorithmic_per_launch": {"flops": flops, "bytes": byts}}
+            "unit": "GB/s", "frac": round(ach / peak, 4), "peak_note": f"{peaks['source']} HBM copy"}
+
+
+def kernel_table(p, prof, gbs, phase, columns, peaks):
+    """Per-kind calls, time, share and roofline fraction of one profiled pass."""
+    out = {}
+    total = sum(v[0] for v in prof.values()) or 1.0
+    for kind, (kms, calls) in prof.items():
+        if calls == 0:
+            continue
+        byts, flops = phase_work(p, kind, calls, gbs, phase, columns)
+        rl = roofline(kind, byts, flops, kms / 1e3, peaks)
+        out[kind] = {"calls": calls, "ms": round(kms, 3), "share": round(kms / total, 4),
+                     "avg_us": round(kms / calls * 1e3, 2), "bound": rl["bound"],
+                     "achieved": rl["achieved"], "unit": rl["unit"], "frac": rl["frac"],
+                     "algorithmic_bytes_per_call": round(byts / calls),
+                     "algorithmic_flops_per_call": round(flops / calls)}
+    return out
+
+
+def codec_rates(fq, torch, p, stream, reps=5):
+    """GB/s of the quantize/pack kernels (weights: fp16 in, packed 4-bit out;
+    2 + 0.5625 bytes per element) and of the dequantizer (0.5625 + 2), on a
+    matrix of the workload's FC1 shape [ffn][h], CUDA events on `stream`."""
+    n_out, k_in = p["ffn"], p["h"]
+    n = n_out * k_in
+    w = torch.empty(n, dtype=torch.float16, device="cuda")
+    fq.flexq_synth_normal_f16(w, n, synth.config_seed(p), synth.TID_TEST_BASE + 99, 0, 0.02, 0.0, stream)
+    packed = torch.empty(fq.flexq_packed_weight_bytes(n_out, k_in), dtype=torch.uint8, device="cuda")
+    codes = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    mn = torch.empty(n // 64, dtype=torch.float16, device="cuda")
+    sc = torch.empty(n // 64, dtype=torch.float16, device="cuda")
+    out = torch.empty_like(w)
+    ops = {
+        "quantize_weight_q4": (lambda: fq.flexq_quantize_weight_q4(w, n_out, k_in, packed, stream), 2.5625),
+        "quantize": (lambda: fq.flexq_quantize(w, n, codes, mn, sc, stream), 2.5625),
+        "dequantize": (lambda: fq.flexq_dequantize(codes, mn, sc, n, out, stream), 2.5625),
+    }
+    res = {}
+    for name, (fn, bpe) in ops.items():
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        stream.synchronize()
+        t = e0.elapsed_time(e1) / reps / 1e3
+        res[name] = {"elements": n, "us": round(t * 1e6, 1), "GBps": round(n * bpe / t / 1e9, 1),
+                     "frac": round(n * bpe / t / 1e9 / load_peaks()["hbm_gbs"], 4)}
+    fq.flexq_device_status(stream)
+    del w, packed, codes, mn, sc, out
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -435,26 +512,21 @@ def run_flexq(args, p):
     step()
     prof = fq.flexq_profile_stop(stream)
     peaks = load_peaks()
-    L_avg = s + n / 2.0
-    kernels = {}
-    total = sum(v[0] for v in prof.values())
-    for kind, (kms, calls) in prof.items():
-        if calls == 0:
-            continue
-        # rows per call: one GPU batch inside the layer steps, the whole block
-        # for the embedding, LM head and argmax (the final LayerNorm's b rows
-        # are counted at the GPU-batch size, which equals b in the default run)
-        M = gbs if kind in ("qkv", "out_proj", "fc1", "fc2", "attn_decode", "kv_append",
-                            "layernorm") else b
-        rl = roofline(p, kind, calls, kms, M, L_avg, peaks)
-        kernels[kind] = {"calls": calls, "ms": round(kms, 3), "share": round(kms / total, 4),
-                         "avg_us": round(kms / calls * 1e3, 2), "bound": rl["bound"],
-                         "achieved": rl["achieved"], "unit": rl["unit"], "frac": rl["frac"]}
+    kernels = kernel_table(p, prof, gbs, "decode", n - 1, peaks)
     dom = max(kernels, key=lambda k: kernels[k]["ms"])
-    rl = roofline(p, dom, prof[dom][1], prof[dom][0], gbs, L_avg, peaks)
+    byts, flops = phase_work(p, dom, prof[dom][1], gbs, "decode", n - 1)
+    rl = roofline(dom, byts, flops, prof[dom][0] / 1e3, peaks)
     rl["traffic"] = ncu_traffic(dom)
-    rl.pop("algorithmic_per_launch", None)
+    rl["algorithmic_per_launch"] = {"bytes": round(byts / prof[dom][1]), "flops": round(flops / prof[dom][1])}
     ceil = step_ceilings(p, gbs, peaks)
+
+    # the prefill column once more, every kernel bracketed
+    fq.flexq_profile_start()
+    fq.flexq_generate_prefill(dm.struct, prompts, b, s, n, gbs, out, ws, ws_n, stream)
+    prof_pre = fq.flexq_profile_stop(stream)
+    fq.flexq_device_status(stream)
+    prefill_kernels = kernel_table(p, prof_pre, gbs, "prefill", 1, peaks)
+    codec = None if args.no_codec else codec_rates(fq, torch, p, stream)
 
     # end to end through flexq_generate: prompts from pinned host memory,
     # tokens back to pinned host memory, all inside the timed region
@@ -507,6 +579,7 @@ def run_flexq(args, p):
             "kernels": kernels,
             "prefill": {"ms": round(prefill_ms, 2),
                         "tokens_per_s": round(world * b * s / (prefill_ms / 1e3), 1),
+                        "kernels": prefill_kernels,
                         "frac_of_ceiling": round(world * b * s / (prefill_ms / 1e3)
                                                  / (world * ceil["prefill_tokens_per_s"]), 4)},
             "ceiling": {"decode_tokens_per_s": round(world * ceil["decode_tokens_per_s"], 1),
@@ -515,6 +588,7 @@ def run_flexq(args, p):
                         "what": "every launched kernel at its own roofline (algorithmic bytes at the "
                                 "measured HBM copy rate or flops at the measured sustained dense rate, "
                                 "whichever is slower), summed over the step"},
+            "codec": codec,
             "gpu_launches": int(launches),
             "gpu_launches_per_step": int(launches // max(1, args.steps)),
             "clocks": clocks,
@@ -539,6 +613,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-codec", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

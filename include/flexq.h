@@ -151,13 +151,15 @@ flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_b
  * (the framework's pool owning the rest of device memory), or a loop that
  * must not pay for cudaMalloc/cudaFree, has no workspace to offer; here the
  * K-split partial sums live in an 8 MiB array compiled into the library
- * (reserved on every GPU that loads it until exit).  Arguments and results
- * as flexq_linear, without ws.  Limit: the K-split scratch the shape needs
- * (flexq_linear_workspace with the same force_splits) must fit in 8 MiB;
- * larger requests return FLEXQ_ERR_INVALID without launching.  The first
- * call on a device looks up the array's address for that device: make it
- * before any stream capture.  All calls share the array (each clears what it
- * uses first); calls that overlap on the GPU race on it, so serialise them.
+ * (reserved on a GPU from the library's first use there until exit).
+ * Arguments and results as flexq_linear, without ws; the output is bit for
+ * bit that of flexq_linear with the same force_splits.  Limit: the K-split
+ * scratch the shape needs (flexq_linear_workspace with the same force_splits)
+ * must fit in 8 MiB; larger requests return FLEXQ_ERR_INVALID without
+ * launching.  The first call on a device looks up the array's address for
+ * that device (kept once found, retried after a failure): make it before any
+ * stream capture.  All calls share the array (each clears what it uses
+ * first); calls that overlap on the GPU race on it, so serialise them.
  * Allocates nothing. */
 flexq_status flexq_linear_static_scratch(const void* x_dev, int ldx, const void* w_dev, int w_bits,
                                          int m, int n, int k, const void* bias_dev,

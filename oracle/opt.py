@@ -31,7 +31,16 @@ reason in the design notes):
 * prefill attends over the K/V of the pass before they are stored; decode
   first appends the new token's K/V (rounded to fp16, then quantized in 4-bit
   mode) and attends over the cached slots 0..pos read back (dequantized);
-* greedy decoding takes the lowest index among equal maxima.
+* greedy decoding takes the lowest index among equal maxima;
+* ``Config.ln1_f16`` (off by default): the LN1 output is rounded to fp16
+  before the Q/K/V projection.  The pages have the layer compute on FP16
+  tensors ("FlexGen研究学术报告" section 三(C): dequantized to FP16 before
+  compute), so the projection's input is an fp16 row there; with the option
+  on, the K/V rows whose 4-bit codes the cache decides come from that same
+  fp16 input.  Every other step stays float64.  A quantization decision is a
+  step function of its input, so where a layer output hangs on those codes the
+  oracle must take them from the input a fp16 layer sees; the GPU parity tests
+  therefore turn the option on for every shape.
 Linear weights are stored [N_out][K_in], so a linear layer is y = x W^T + b.
 """
 from __future__ import annotations
@@ -56,15 +65,17 @@ class Config:
     w_bits: int = 4
     kv_bits: int = 4
     eps: float = 1e-5
+    ln1_f16: bool = False
 
     @property
     def d(self) -> int:
         return self.h // self.heads
 
     @staticmethod
-    def from_preset(p: dict) -> "Config":
+    def from_preset(p: dict, ln1_f16: bool = False) -> "Config":
         return Config(layers=p["layers"], h=p["h"], heads=p["heads"], ffn=p["ffn"],
-                      vocab=p["vocab"], w_bits=p["w_bits"], kv_bits=p["kv_bits"])
+                      vocab=p["vocab"], w_bits=p["w_bits"], kv_bits=p["kv_bits"],
+                      ln1_f16=ln1_f16)
 
 
 # ---------------------------------------------------------------------------
@@ -239,6 +250,13 @@ def attention_single(q, k, v):
 # ---------------------------------------------------------------------------
 # Layer
 # ---------------------------------------------------------------------------
+def projection_input(cfg, W, x):
+    """u = LN1(x), rounded to fp16 when cfg.ln1_f16 (the projection input of
+    a layer that computes in fp16)."""
+    u = layernorm(x, W["ln1_g"], W["ln1_b"], cfg.eps)
+    return f16(u) if cfg.ln1_f16 else u
+
+
 def _mlp(cfg, W, x_out):
     v = layernorm(x_out, W["ln2_g"], W["ln2_b"], cfg.eps)
     g = gelu(linear(v, W["w_fc1"], W["b_fc1"]))
@@ -249,7 +267,7 @@ def layer_prefill(cfg: Config, W: dict, x: np.ndarray):
     """x: [b, s, h] -> (y [b, s, h], K16 [b, s, h], V16 [b, s, h]).  K16/V16
     are the fp16-rounded keys/values the cache stores for slots 0..s-1."""
     h = cfg.h
-    u = layernorm(x, W["ln1_g"], W["ln1_b"], cfg.eps)
+    u = projection_input(cfg, W, x)
     qkv = linear(u, W["w_qkv"], W["b_qkv"])
     Q, K, V = qkv[..., :h], qkv[..., h:2 * h], qkv[..., 2 * h:]
     a = cfg.heads
@@ -263,7 +281,7 @@ def layer_decode(cfg: Config, W: dict, t: np.ndarray, cache: KVCache, pos: int):
     """t: [b, h] (the token at position pos) -> t' [b, h].  Appends this
     token's K/V to slot pos of the cache, then attends over slots 0..pos."""
     h, a = cfg.h, cfg.heads
-    u = layernorm(t, W["ln1_g"], W["ln1_b"], cfg.eps)
+    u = projection_input(cfg, W, t)
     qkv = linear(u, W["w_qkv"], W["b_qkv"])
     Q, K, V = qkv[:, :h], qkv[:, h:2 * h], qkv[:, 2 * h:]
     cache.write("k", K.astype(np.float16)[:, None, :], pos)

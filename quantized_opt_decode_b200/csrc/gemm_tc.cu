@@ -11,40 +11,22 @@
 //
 // One output tile = 128 features x up to 256 tokens; the weight is the MMA's A
 // operand, so a small decode batch becomes the MMA's N.  A persistent CTA per
-// SM walks a list of (tile, k-block range) segments.  Two kernels share the
-// scheduler and the epilogue:
-//
-// gemm_w4_decode_kernel (4-bit weights, decode-sized token tiles <= 160 whose K
-// has an odd number of 64-wide k-blocks):
-//   warp 0      TMA producer: per 64-wide k-block one cp.async.bulk of the
-//               packed chunk (codes + min/scale, 4608 contiguous bytes) and
-//               one 128-byte-swizzled cp.async.bulk.tensor of the activations
-//               into a deep shared-memory ring;
-//   warps 2-9   two dequantizing warpgroups taking alternate k-blocks.  Each
-//               thread turns one weight row of the k-block into fp16
-//               ((code | 0x6400) is the fp16 value 1024 + code; one half2
-//               subtract and one half2 fused multiply-add give
-//               code * scale + min rounded once) and stores it straight into
-//               tensor memory (tcgen05.st): no shared-memory round trip for
-//               A.  A named barrier closes the group's step and one thread
-//               signals it with a single mbarrier arrival.  Each group has
-//               its own A ring in tensor memory, so the two groups' steps
-//               overlap;
-//   warp 1      owns TMEM and, from one thread, issues the k-blocks'
-//               tcgen05.mma.kind::f16 (M=128, N=tokens, K=16, A from tensor
-//               memory) x 4 in k order, alternating between the groups' rings.
-//               The issuing thread stalls while the tensor pipe's queue is
-//               full; keeping it out of the dequantizing warps keeps that
-//               stall off their critical path;
+// SM walks a list of (tile, k-block range) segments:
+//   warp 0      TMA producer: per pipeline stage one cp.async.bulk of the
+//               packed weight chunks (codes + min/scale, 4608 contiguous bytes
+//               per 64-wide k-block) and one 128-byte-swizzled
+//               cp.async.bulk.tensor box of the activations per k-block;
+//   warps 2-9   dequantize the weight rows into a shared-memory ring of fp16
+//               A tiles in the UMMA K-major SW128 layout ((code | 0x6400) is
+//               the fp16 value 1024 + code; one half2 subtract and one half2
+//               fused multiply-add give code * scale + min rounded once);
+//   warp 1      owns TMEM and, from one thread, issues tcgen05.mma.kind::f16
+//               (M=128, N=tokens, K=16; A and B from shared memory);
 //   warps 10-13 epilogue (below).
-//
-// gemm_tc_kernel (everything else: prefill-sized tiles, fp16 weights, and
-// decode-sized 4-bit tiles with an even number of k-blocks, which it moves two
-// k-blocks per pipeline stage; on the OPT-30B decode shapes this measured
-// faster than the tensor-memory-A kernel):
-//   warp 0 TMA producer; warps 2-9 dequantize into a shared-memory ring of
-//   fp16 A tiles in the UMMA K-major SW128 layout; warp 1 issues the MMAs from
-//   one thread (A and B from shared memory); warps 10-13 epilogue.
+// Decode-sized tiles (<= 160 tokens) on 4-bit weights move two k-blocks per
+// stage when K allows (half the mbarrier hand-offs per FLOP); fp16 weights
+// (the LM head, fp16-weight configurations) arrive by TMA and skip the
+// dequantizing warps.
 //
 // Epilogue (warps 10-13, one TMEM lane quarter each): tcgen05.ld, + bias,
 // GELU, + residual, fp16 or fp32 store; two accumulator buffers let it overlap
@@ -70,7 +52,6 @@ namespace {
 
 constexpr int kThreads = 448;
 constexpr int kDequantThreads = 256;
-constexpr int kGroupThreads = 128;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
 constexpr int kATileBytes = 128 * 64 * 2;
@@ -105,7 +86,6 @@ struct GemmParams {
   uint32_t load_stage_bytes;
   uint32_t acc_cols;    // TMEM columns between the two accumulator buffers
   uint32_t tmem_alloc;  // columns allocated (power of two)
-  uint32_t a_col0;      // first TMEM column of the A rings (decode kernel)
   Sched sc;
   const __half* bias;
   const __half* residual;
@@ -502,7 +482,7 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
   }
 }
 
-// Teardown shared by both kernels: free TMEM once every thread is done (the
+// Teardown: free TMEM once every thread is done (the
 // MMA-issuing threads have waited for their own MMAs before getting here).
 __device__ __forceinline__ void teardown(const GemmParams& p, const Ctl& c, uint32_t tmem_base, int warp) {
   tc_fence_before();
@@ -511,202 +491,6 @@ __device__ __forceinline__ void teardown(const GemmParams& p, const Ctl& c, uint
     tc_fence_after();
     tmem_dealloc(tmem_base, p.tmem_alloc);
   }
-}
-
-// ---------------------------------------------------------------------------
-// decode kernel: 4-bit weights, A dequantized into tensor memory by two
-// warpgroups; one thread issues the MMAs
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_w4_decode_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
-  extern __shared__ uint8_t smem_dyn[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  const int SL = p.load_stages, SA = p.a_stages;  // SA: A slots per group
-  uint8_t* l_ring = smem;                         // SL x [activation box | raw chunk]
-  uint8_t* region = l_ring + SL * p.load_stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(region);
-  uint64_t* empty = full + SL;
-  uint64_t* afull = empty + SL;        // [2][SA] A slot written (one arrival per group step)
-  uint64_t* aempty = afull + 2 * SA;   // [2][SA] A slot consumed by its MMAs
-  uint64_t* drained = aempty + 2 * SA; // the MMA thread's final drain
-  const Ctl c = make_ctl(region, drained + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int cta = blockIdx.x;
-  const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < SL; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < 2 * SA; ++s) {
-      mbar_init(&afull[s], 1);
-      mbar_init(&aempty[s], 1);
-    }
-    mbar_init(drained, 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&c.accf[b], 1);
-      mbar_init(&c.acce[b], kEpiThreads);
-    }
-    *c.abort_flag = 0;
-    mbar_fence_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(c.tmem_slot, p.tmem_alloc);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *c.tmem_slot;
-  const Sched& sc = p.sc;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tmap_x);
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
-      const uint32_t tx_bytes = static_cast<uint32_t>(kTileBytes) + b_bytes;
-      int i = 0;
-      Ring rl;
-      Seg g;
-      bool stop = false;
-      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-        const int n_tile = g.tile % sc.n_tiles;
-        const int t_row = (g.tile / sc.n_tiles) * p.tok_tile;
-        const uint8_t* wsrc = p.wq + (static_cast<size_t>(n_tile) * p.kb_real + g.kb0) * kTileBytes;
-        for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL), wsrc += kTileBytes) {
-          const int s = rl.s;
-          if (!mbar_wait(&empty[s], rl.ph ^ 1u, p.wait_ns)) {
-            set_error(p.err, DEV_TIMEOUT_PRODUCER);
-            *c.abort_flag = 1;
-          }
-          if (*c.abort_flag) {
-            stop = true;
-            break;
-          }
-          uint8_t* st = l_ring + s * p.load_stage_bytes;
-          mbar_arrive_expect_tx(&full[s], tx_bytes);
-          bulk_load(st + b_bytes, wsrc, kTileBytes, &full[s], pol_w);
-          tma_load_2d(st, &tmap_x, &full[s], ks * 64, t_row, pol_x);
-        }
-      }
-      // Never leave the CTA with bulk copies still landing in its shared memory.
-      for (int j = max(0, i - SL); j < i; ++j)
-        mbar_wait(&full[j % SL], static_cast<uint32_t>(j / SL) & 1u, drain_ns(p.wait_ns));
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
-      const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(l_ring));
-      const uint32_t l_step = p.load_stage_bytes >> 4;
-      Ring rl, ra[2];
-      int i = 0;  // k-block index over all segments; group i & 1 dequantized it
-      Seg g;
-      bool stop = false;
-      for (int q = 0; get_seg(sc, cta, q, g); ++q) {
-        int buf;
-        uint32_t par;
-        acc_slot(q, buf, par);
-        if (!stop && !mbar_wait(&c.acce[buf], par ^ 1u, p.wait_ns)) {
-          set_error(p.err, DEV_TIMEOUT_MMA);
-          *c.abort_flag = 1;
-        }
-        if (*c.abort_flag) stop = true;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols;
-        for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, ++i, rl.next(SL)) {
-          const int grp = i & 1;
-          const int slot = grp * SA + ra[grp].s;
-          if (!mbar_wait(&afull[slot], ra[grp].ph, p.wait_ns)) {
-            set_error(p.err, DEV_TIMEOUT_MMA);
-            *c.abort_flag = 1;
-          }
-          if (*c.abort_flag) {
-            stop = true;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_tmem = tmem_base + p.a_col0 + static_cast<uint32_t>(slot) * 32u;
-          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(rl.s * l_step);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_f16_ts(d_tmem, a_tmem + 8 * kk, bdesc + 2 * kk, idesc, (ks > g.kb0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[rl.s]);
-          mma_commit(&aempty[slot]);
-          ra[grp].next(SA);
-        }
-        // Every segment ends with a commit, also after an abort, so the
-        // epilogue never waits on a barrier nobody signals.
-        mma_commit(&c.accf[buf]);
-      }
-      // all MMAs have completed before TMEM can be released
-      mma_commit(drained);
-      mbar_wait(drained, 0, drain_ns(p.wait_ns));
-    }
-  } else if (warp < kEpiWarp0) {
-    // ------------------------------------------------------------ dequantize
-    const int grp = (warp - 2) >> 2;
-    const int quarter = warp & 3;  // TMEM lanes this warp may store to
-    const int row = quarter * 32 + lane;
-    const bool signaller = lane == 0 && warp == 2 + 4 * grp;
-    const uint32_t t_row = tmem_base + p.a_col0 + static_cast<uint32_t>(grp * SA) * 32u +
-                           (static_cast<uint32_t>(quarter * 32) << 16);
-    int i = 0;  // k-block index over all segments of this CTA (both groups)
-    Ring rl, ra;
-    bool stop = false;
-    Seg g;
-    for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-      for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL)) {
-        if ((i & 1) != grp) continue;
-        const int s = rl.s;
-        const int a = ra.s;
-        bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
-        ok = ok && mbar_wait(&aempty[grp * SA + a], ra.ph ^ 1u, p.wait_ns);
-        if (!ok) {
-          set_error(p.err, DEV_TIMEOUT_CONSUMER);
-          *c.abort_flag = 1;
-        }
-        tc_fence_after();
-        // this thread's weight row of the k-block: 64 codes + (min, scale)
-        const uint8_t* raw = l_ring + s * p.load_stage_bytes + b_bytes;
-        const uint4 w0 = *reinterpret_cast<const uint4*>(raw + row * 32);
-        const uint4 w1 = *reinterpret_cast<const uint4*>(raw + row * 32 + 16);
-        const __half2 mm = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
-        const __half2 m2 = __low2half2(mm);
-        const __half2 s2 = __high2half2(mm);
-        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        uint32_t r[32];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint4 d = dequant8(words[j], s2, m2);
-          r[4 * j] = d.x;
-          r[4 * j + 1] = d.y;
-          r[4 * j + 2] = d.z;
-          r[4 * j + 3] = d.w;
-        }
-        __syncwarp();
-        tmem_st_x32(t_row + static_cast<uint32_t>(a) * 32u, r);
-        tmem_st_wait();
-        tc_fence_before();
-        // the whole group has stored its rows (or someone gave up)
-        if (bar_any<kGroupThreads>(2 + grp, !ok || *c.abort_flag)) {
-          stop = true;
-          break;
-        }
-        if (signaller) mbar_arrive(&afull[grp * SA + a]);
-        ra.next(SA);
-      }
-    }
-  } else {
-    epilogue_role(p, c, tmem_base, warp, lane);
-  }
-  teardown(p, c, tmem_base, warp);
 }
 
 // ---------------------------------------------------------------------------
@@ -941,7 +725,7 @@ EncodeTiledFn encode_fn() {
 
 // 2-D fp16 tensor [rows][cols] with row stride ld (elements), box 64 x box_rows,
 // 128-byte swizzle, zero fill out of bounds.
-bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
+bool encode_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
@@ -953,14 +737,51 @@ bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Encoded maps keyed by everything that goes into them, so repeated calls on
+// the same buffers (every decode step) skip the encoding.  A map holds only
+// the address, extents, stride and box, so a key always yields the same map.
+struct TmapKey {
+  const void* base;
+  int rows, cols, ld, box_rows;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows;
+  }
+};
+constexpr int kTmapCache = 64;
+struct TmapCache {
+  std::mutex mu;
+  TmapKey key[kTmapCache];
+  CUtensorMap map[kTmapCache];
+  bool used[kTmapCache] = {};
+  int next = 0;
+};
+TmapCache g_tmaps;
+
+bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
+  const TmapKey k{base, rows, cols, ld, box_rows};
+  std::lock_guard<std::mutex> lock(g_tmaps.mu);
+  for (int i = 0; i < kTmapCache; ++i) {
+    if (g_tmaps.used[i] && g_tmaps.key[i] == k) {
+      *map = g_tmaps.map[i];
+      return true;
+    }
+  }
+  if (!encode_tmap(map, base, rows, cols, ld, box_rows)) return false;
+  const int i = g_tmaps.next;
+  g_tmaps.next = (i + 1) % kTmapCache;
+  g_tmaps.key[i] = k;
+  g_tmaps.map[i] = *map;
+  g_tmaps.used[i] = true;
+  return true;
+}
+
 struct Plan {
   int tok_tile, tok_tiles, n_tiles;
-  bool decode;  // gemm_w4_decode_kernel
   int ks;       // k-blocks per stage of gemm_tc_kernel
   Sched sc;
   int load_stages, a_stages;
   uint32_t load_stage_bytes;
-  uint32_t acc_cols, tmem_alloc, a_col0;
+  uint32_t acc_cols, tmem_alloc;
   size_t smem;
   size_t partial_bytes, counter_bytes;
 };
@@ -982,13 +803,10 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.tok_tile = round_up((m + P.tok_tiles - 1) / P.tok_tiles, 16);
   }
   // Decode-sized tiles on 4-bit weights: two k-blocks per shared-memory stage
-  // (measured fastest on the OPT-30B decode shapes).  Where K has an odd
-  // number of k-blocks two per stage do not divide it, and the tensor-memory-A
-  // kernel takes the shape (its speed against one k-block per stage in the
-  // shared-memory kernel is unmeasured; every benchmark shape has even K/64).
+  // where K has an even number of k-blocks (measured fastest on the OPT-30B
+  // decode shapes; every benchmark shape has even K/64).
   const bool dec = w_bits == 4 && P.tok_tile <= kDecodeMaxTok;
   P.ks = dec && kb_real % 2 == 0 ? 2 : 1;
-  P.decode = dec && P.ks == 1;
   const int kb_total = kb_real / P.ks;  // k-steps per tile
   const int min_iters = max(1, kMinItersPerCta / P.ks);
   P.n_tiles = (n + 127) / 128;
@@ -1028,15 +846,7 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
   const int b_bytes = P.tok_tile * 128;
   int a_slot = 0;
-  if (P.decode) {
-    // TMEM: two accumulator buffers, then one A ring per group (32 columns =
-    // 128 rows x 64 fp16 per slot)
-    P.acc_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
-    P.a_col0 = 2 * P.acc_cols;
-    P.tmem_alloc = 512;
-    P.a_stages = min(4, static_cast<int>((512 - P.a_col0) / 64));
-    P.load_stage_bytes = static_cast<uint32_t>(b_bytes + kRawStageBytes);
-  } else {
+  {
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
     P.acc_cols = cols;
@@ -1077,13 +887,6 @@ cudaError_t launch_general(const Plan& P, const CUtensorMap& tx, const CUtensorM
   return launched();
 }
 
-cudaError_t launch_decode(const Plan& P, const CUtensorMap& tx, const GemmParams& p, cudaStream_t s) {
-  const cudaError_t e = configure_once<gemm_w4_decode_kernel>();
-  if (e != cudaSuccess) return e;
-  gemm_w4_decode_kernel<<<P.sc.grid, kThreads, P.smem, s>>>(tx, p);
-  return launched();
-}
-
 }  // namespace
 
 size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits) {
@@ -1098,9 +901,9 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   const bool w4 = a.w_bits == 4;
   if (P.load_stages < 2) return cudaErrorInvalidValue;
   // mbarriers the kernel lays out before its control words (make_ctl):
-  // decode: full/empty per load stage, afull/aempty per A slot of each group,
-  // the drain barrier, accf/acce x 2; general: the same with one A ring
-  const int n_bars = P.decode ? 2 * P.load_stages + 4 * P.a_stages + 5 : 2 * P.load_stages + 2 * P.a_stages + 5;
+  // full/empty per load stage, afull/aempty per A slot, the drain barrier,
+  // accf/acce x 2
+  const int n_bars = 2 * P.load_stages + 2 * P.a_stages + 5;
   if (n_bars > kMaxBarriers) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
   if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile)) return cudaErrorInvalidValue;
@@ -1121,7 +924,6 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.load_stage_bytes = P.load_stage_bytes;
   p.acc_cols = P.acc_cols;
   p.tmem_alloc = P.tmem_alloc;
-  p.a_col0 = P.a_col0;
   p.sc = P.sc;
   p.bias = a.bias;
   p.residual = a.residual;
@@ -1144,7 +946,6 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
     const cudaError_t e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
     if (e != cudaSuccess) return e;
   }
-  if (P.decode) return launch_decode(P, tx, p, s);
   if (w4 && P.ks == 2) return launch_general<true, 2>(P, tx, tw, p, s);
   if (w4) return launch_general<true, 1>(P, tx, tw, p, s);
   return launch_general<false, 1>(P, tx, tw, p, s);

@@ -13,10 +13,12 @@
 // Properties a user must know:
 // * The array holds kStaticScratchBytes (8 MiB) of fp32 partial tiles; a shape
 //   whose K-split scratch (flexq_linear_workspace) is larger is rejected with
-//   FLEXQ_ERR_INVALID before anything is launched.  Every GPU that loads the
-//   library keeps these 8 MiB reserved until the process exits.
-// * The first call on a device looks up the array's device address (once per
-//   device, with that device current).  Make that first call before any
+//   FLEXQ_ERR_INVALID before anything is launched.  The 8 MiB are reserved
+//   on a device from the first use of the library's device code there (with
+//   lazy module loading, the first launch) until the process exits.
+// * The first call on a device looks up the array's device address (with that
+//   device current) and keeps it once the lookup succeeds; a failed lookup is
+//   reported and retried by the next call.  Make that first call before any
 //   stream capture begins.
 // * All calls share the one array and it keeps the last call's contents; each
 //   call clears the part it uses before accumulating.  Calls whose kernels
@@ -40,25 +42,31 @@ constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDev = 64;
-void* g_scratch_ptr[kMaxDev];
-cudaError_t g_scratch_rc[kMaxDev];
-std::once_flag g_scratch_once[kMaxDev];
+void* g_scratch_ptr[kMaxDev];  // set once the lookup on that device succeeded
+std::mutex g_scratch_mu;
 
 // Device address of the static array on the current device.  In host code the
 // name g_static_scratch is only a host-side stand-in, so the address must come
-// from cudaGetSymbolAddress; this runs once per device.
+// from cudaGetSymbolAddress.  A successful lookup is kept for the device; a
+// failed one (for example during a stream capture) is not, so a later call
+// tries again.
 cudaError_t scratch_on_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  std::call_once(g_scratch_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    g_scratch_rc[dev] = cudaGetSymbolAddress(&p, g_static_scratch);
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // the failure is reported through the return value
+      return e;
+    }
     g_scratch_ptr[dev] = p;
-  });
+  }
   *out = g_scratch_ptr[dev];
-  return g_scratch_rc[dev];
+  return cudaSuccess;
 }
 
 }  // namespace

@@ -77,3 +77,33 @@ def v_words_to_canonical(words: np.ndarray, b: int, heads: int, max_len: int, d:
         codes[:, :, :, k, :] = (w >> np.uint32(4 * k)) & np.uint32(0xF)
     codes = codes.reshape(b, heads, l8, d)[:, :, :max_len]
     return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def ulp16(x):
+    """Spacing of fp16 numbers at |x| (the subnormal spacing below 2^-14)."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 10)
+
+
+def assert_close(got, ref, tol=2e-3, c=10.0, what=""):
+    """The parity bar of the GPU tests: relative Frobenius error below `tol`,
+    and every element within one fp16 ulp of its reference plus c * tol times
+    the reference's rms.  The second bound catches a single wrong element
+    (an indexing slip in one tile) that a norm over 10^6 elements would
+    average away."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    r = rel_fro(got, ref)
+    assert r < tol, f"{what}: relative Frobenius error {r:.3e} >= {tol:.1e}"
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    bound = ulp16(ref) + c * tol * rms
+    err = np.abs(got - ref)
+    excess = err - bound
+    k = int(np.argmax(excess)) if excess.size else 0
+    assert excess.size == 0 or excess.flat[k] <= 0, (
+        f"{what}: element {np.unravel_index(k, ref.shape)} off by {err.flat[k]:.3e} "
+        f"(ref {ref.flat[k]:.4e}, bound {bound.flat[k]:.3e}, rms {rms:.3e})")
+    return r

@@ -1,8 +1,11 @@
 """GPU parity of whole layer steps and of generation against the oracle.
 
 Layer steps (prefill over b x s tokens, then decode of one token) on the tiny
-configuration and on a d = 128 variant, 4-bit and fp16 weights/KV: max relative
-Frobenius error 2e-3 on the layer output, and on the layer's residual branch
+configuration and on a d = 128 variant, 4-bit and fp16 weights/KV, against the
+oracle with the LN1 output rounded to fp16 (the projection input of a layer
+that computes in fp16, as for every shape): max relative Frobenius error 2e-3
+on the layer output and the element-wise bound of gpu_helpers.assert_close,
+and on the layer's residual branch
 (y - x) a bound of 2e-3 relative to the output norm as well.  Cached codes are
 compared element by element: the K/V rows come out of a GEMM on each side, so
 a value sitting on a rounding boundary may land one code apart; at least 99%
@@ -20,7 +23,7 @@ pytestmark = pytest.mark.gpu
 
 import synth  # noqa: E402
 from oracle import opt  # noqa: E402
-from gpu_helpers import fq, rel_fro, to_dev, to_host  # noqa: E402
+from gpu_helpers import assert_close, fq, rel_fro, to_dev, to_host  # noqa: E402
 from quantized_opt_decode_b200.device_model import DeviceModel, workspace  # noqa: E402
 
 TOL = 2e-3
@@ -35,7 +38,7 @@ def _preset(name, **over):
 def _layer_roundtrip(p, b, s):
     """Runs prefill then one decode through layer 0 on both sides."""
     dm = DeviceModel(p, b=b, max_len=s + 4, layers=1)
-    cfg = opt.Config.from_preset(p)
+    cfg = opt.Config.from_preset(p, ln1_f16=True)
     seed = synth.config_seed(p)
     W = opt.effective_layer(cfg, opt.raw_layer(cfg, seed, 0))
     rng = np.random.default_rng(b * s + p["h"])
@@ -61,7 +64,7 @@ def _layer_roundtrip(p, b, s):
 
 
 def _check_out(got, ref, x):
-    assert rel_fro(got, ref) < TOL, rel_fro(got, ref)
+    assert_close(got, ref, TOL)
     branch = np.linalg.norm(got.astype(np.float64) - ref) / np.linalg.norm(ref - x.astype(np.float64))
     assert branch < 1e-2, branch  # error relative to the layer's own contribution
 
@@ -105,7 +108,7 @@ def test_generate_tokens_valid_under_oracle(name):
     fq.flexq_generate(dm.struct, to_dev(prompts), b, s, n, p["gpu_batch"], out, ws, ws_n, timing)
     fq.flexq_device_status()
     toks = to_host(out)
-    m = opt.build_model(opt.Config.from_preset(p), seed, s + n)
+    m = opt.build_model(opt.Config.from_preset(p, ln1_f16=True), seed, s + n)
     own, _ = opt.generate(m, prompts, n)
     _, logits = opt.generate(m, prompts, n, forced=toks)
     for j in range(n):

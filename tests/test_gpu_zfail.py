@@ -8,7 +8,7 @@ import torch
 pytestmark = pytest.mark.gpu
 
 from oracle import q64  # noqa: E402
-from gpu_helpers import fq, rel_fro, to_dev, to_host  # noqa: E402
+from gpu_helpers import assert_close, fq, to_dev, to_host  # noqa: E402
 
 
 def _gemm(m=128, n=1024, k=4096):
@@ -40,7 +40,7 @@ def test_wait_timeout_is_reported_and_context_survives():
         fq.flexq_set_wait_limit_ns(0)
     run()
     fq.flexq_device_status()
-    assert rel_fro(to_host(y), ref) < 2e-3
+    assert_close(to_host(y), ref, 2e-3)
 
 
 def test_bad_token_id_is_reported():

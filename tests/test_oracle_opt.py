@@ -327,3 +327,191 @@ def test_generate_prefill_token_and_teacher_forcing():
 def test_greedy_lowest_index_on_ties():
     lg = np.array([[1.0, 3.0, 3.0, 2.0], [5.0, 5.0, 5.0, 5.0]])
     assert opt.greedy(lg).tolist() == [1, 0]
+
+
+# ---------------------------------------------------------------------------
+# Embedding, tied LM head, group axis and the fp16-LN1 reading, by brute force
+# ---------------------------------------------------------------------------
+def _bf_ln(row, g, b, eps=1e-5):
+    mu = sum(row) / len(row)
+    var = sum((t - mu) ** 2 for t in row) / len(row)
+    return [(t - mu) / math.sqrt(var + eps) * float(g[i]) + float(b[i]) for i, t in enumerate(row)]
+
+
+def _bf_lin(row, w, b):
+    return [sum(row[k] * float(w[n][k]) for k in range(len(row))) + float(b[n]) for n in range(len(w))]
+
+
+def test_embed_brute_force():
+    """x0[i][t] = E[tok[i][t]] + P[t] element by element from the fp16 tables
+    (survey notes: word embedding plus positional embedding)."""
+    cfg = opt.Config(layers=1, h=128, heads=2, ffn=256, vocab=40, w_bits=4, kv_bits=4)
+    m = opt.build_model(cfg, 77, 9)
+    tok = np.array([[3, 0, 39, 3], [12, 12, 7, 38]])
+    pos = np.arange(4)[None, :] + np.array([[0], [5]])
+    got = opt.embed(m, tok, pos)
+    for i in range(2):
+        for t in range(4):
+            for e in range(cfg.h):
+                want = float(m.E[tok[i, t]][e]) + float(m.P[pos[i, t]][e])
+                assert got[i, t, e] == want
+    # the word and the position rows are distinct tables, not swapped
+    assert not np.array_equal(opt.embed(m, tok[:, :1], pos[:, 1:2]), opt.embed(m, tok[:, 1:2], pos[:, :1]))
+
+
+def test_lm_logits_brute_force():
+    """logits[i][v] = sum_e LN_f(x_i)[e] * E[v][e]: final LayerNorm, then the
+    word-embedding matrix as the LM head ("内存占用分析": tied embedding)."""
+    cfg = opt.Config(layers=1, h=128, heads=2, ffn=256, vocab=24, w_bits=4, kv_bits=4)
+    m = opt.build_model(cfg, 78, 4)
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((2, cfg.h)) * 2 + 0.3
+    got = opt.lm_logits(m, x)
+    for i in range(2):
+        u = _bf_ln(x[i].tolist(), m.lnf_g, m.lnf_b)
+        for v in range(cfg.vocab):
+            want = sum(u[e] * float(m.E[v][e]) for e in range(cfg.h))
+            assert math.isclose(got[i, v], want, rel_tol=1e-11, abs_tol=1e-11)
+
+
+def test_effective_layer_groups_run_along_k_in():
+    """A weight that is constant over every 64-wide span of K_in inside a row
+    (and varies across rows) is reproduced exactly: each group is constant, so
+    scale 0 and x_hat = min.  Groups taken along N_out (the transposed memory
+    order) would mix 64 different rows and could not be exact."""
+    cfg = opt.Config(layers=1, h=128, heads=2, ffn=256, vocab=8, w_bits=4, kv_bits=4)
+    rng = np.random.default_rng(9)
+    raw = opt.raw_layer(cfg, 5, 0)
+    for name in opt.LINEAR:
+        n, k = raw[name].shape
+        c = rng.standard_normal((n, k // 64)).astype(np.float16)
+        raw[name] = np.repeat(c, 64, axis=1)
+    eff = opt.effective_layer(cfg, raw)
+    for name in opt.LINEAR:
+        assert np.array_equal(eff[name], raw[name].astype(np.float64)), name
+        assert not np.array_equal(q64.roundtrip(raw[name].T.copy()).T, raw[name])
+
+
+def _bf_decode(cfg, W, t, keys, values, ln1_f16):
+    """One decode step for one sequence written out as loops: keys/values are
+    the cached rows [L][h] of slots 0..pos-1 (float values as read back); the
+    new token's K/V (fp16-rounded) is appended last.  Returns (t', K_new)."""
+    h, a, d = cfg.h, cfg.heads, cfg.d
+    u = _bf_ln(t, W["ln1_g"], W["ln1_b"])
+    if ln1_f16:
+        u = [float(np.float16(v)) for v in u]
+    qkv = _bf_lin(u, W["w_qkv"], W["b_qkv"])
+    q = qkv[:h]
+    k_new = [float(np.float16(v)) for v in qkv[h:2 * h]]
+    v_new = [float(np.float16(v)) for v in qkv[2 * h:]]
+    K, V = keys + [k_new], values + [v_new]
+    o = [0.0] * h
+    for j in range(a):
+        sl = slice(j * d, (j + 1) * d)
+        z = bf_attention([q[sl]], [r[sl] for r in K], [r[sl] for r in V], False)[0]
+        o[j * d:(j + 1) * d] = z
+    xo = [p + r for p, r in zip(_bf_lin(o, W["w_o"], W["b_o"]), t)]
+    v2 = _bf_ln(xo, W["ln2_g"], W["ln2_b"])
+    f1 = [z * 0.5 * (1 + math.erf(z / math.sqrt(2))) for z in _bf_lin(v2, W["w_fc1"], W["b_fc1"])]
+    return [p + r for p, r in zip(_bf_lin(f1, W["w_fc2"], W["b_fc2"]), xo)], k_new
+
+
+@pytest.mark.parametrize("ln1_f16", [False, True])
+def test_decode_brute_force_fp16_kv(ln1_f16):
+    """16-bit KV decode (append fp16(K), attend over slots 0..pos) against
+    loops, with and without the fp16 rounding of the LN1 output; the two
+    readings are different functions (the option is not a no-op)."""
+    cfg = opt.Config(layers=1, h=128, heads=2, ffn=128, vocab=8, w_bits=16, kv_bits=16, ln1_f16=ln1_f16)
+    W = rand_layer(cfg, seed=11)
+    rng = np.random.default_rng(12)
+    pos = 3
+    hist = rng.standard_normal((1, pos, cfg.h)).astype(np.float16)
+    cache = opt.KVCache(cfg, 1, pos + 1, 16)
+    cache.write("k", hist, 0)
+    cache.write("v", hist * np.float16(0.5), 0)
+    t = rng.standard_normal((1, cfg.h))
+    got = opt.layer_decode(cfg, W, t, cache, pos)
+    keys = hist[0].astype(np.float64).tolist()
+    vals = (hist[0] * np.float16(0.5)).astype(np.float64).tolist()
+    want, k_new = _bf_decode(cfg, W, t[0].tolist(), keys, vals, ln1_f16)
+    assert np.allclose(got[0], want, rtol=1e-10, atol=1e-10)
+    assert cache.t["k"][0, :, pos].reshape(-1).astype(np.float64).tolist() == k_new
+    other = opt.Config(**{**cfg.__dict__, "ln1_f16": not ln1_f16})
+    cache2 = opt.KVCache(other, 1, pos + 1, 16)
+    cache2.write("k", hist, 0)
+    cache2.write("v", hist * np.float16(0.5), 0)
+    assert not np.array_equal(opt.layer_decode(other, W, t, cache2, pos), got)
+
+
+def _bf_dequant_slot(cache, kv, i, pos):
+    """Slot `pos` of sequence i read back from the 4-bit cache by loops over
+    the nibbles: x_hat = fp16(fp32(code * scale) + min), low nibble = even
+    element, one (min, scale) pair per 64 elements of a head row."""
+    cfg = cache.cfg
+    row = []
+    for j in range(cfg.heads):
+        codes = cache.t[kv + "_codes"][i, j, pos]
+        for e in range(cfg.d):
+            byte = int(codes[e // 2])
+            q = byte & 15 if e % 2 == 0 else byte >> 4
+            g = e // 64
+            s = np.float32(cache.t[kv + "_scale"][i, j, pos, g])
+            m = np.float32(cache.t[kv + "_min"][i, j, pos, g])
+            row.append(float(np.float16(np.float32(np.float32(q) * s) + m)))
+    return row
+
+
+@pytest.mark.parametrize("ln1_f16", [False, True])
+def test_decode_brute_force_4bit_kv(ln1_f16):
+    """4-bit KV decode against loops that read every cached element back from
+    its nibble and its group's (min, scale): pins the dequantizing read path
+    and the attention over slots 0..pos (including the appended slot) to
+    1e-10, far tighter than a prefill/decode comparison can."""
+    cfg = opt.Config(layers=1, h=128, heads=2, ffn=128, vocab=8, w_bits=4, kv_bits=4, ln1_f16=ln1_f16)
+    W = rand_layer(cfg, seed=13)
+    rng = np.random.default_rng(14)
+    pos = 4
+    cache = opt.KVCache(cfg, 1, pos + 2, 4)
+    cache.write("k", rng.standard_normal((1, pos, cfg.h)).astype(np.float16), 0)
+    cache.write("v", rng.standard_normal((1, pos, cfg.h)).astype(np.float16), 0)
+    t = rng.standard_normal((1, cfg.h))
+    got = opt.layer_decode(cfg, W, t, cache, pos)
+    keys = [_bf_dequant_slot(cache, "k", 0, p) for p in range(pos + 1)]
+    vals = [_bf_dequant_slot(cache, "v", 0, p) for p in range(pos + 1)]
+    # the brute force appends its own fp16 K/V row; swap in the cached slot
+    # (its codes are pinned by test_decode_appends_quantized_row) so that the
+    # loop attends over exactly what the cache holds
+    h, a, d = cfg.h, cfg.heads, cfg.d
+    u = _bf_ln(t[0].tolist(), W["ln1_g"], W["ln1_b"])
+    if ln1_f16:
+        u = [float(np.float16(v)) for v in u]
+    qkv = _bf_lin(u, W["w_qkv"], W["b_qkv"])
+    o = [0.0] * h
+    for j in range(a):
+        sl = slice(j * d, (j + 1) * d)
+        o[sl] = bf_attention([qkv[:h][sl]], [r[sl] for r in keys], [r[sl] for r in vals], False)[0]
+    xo = [p + r for p, r in zip(_bf_lin(o, W["w_o"], W["b_o"]), t[0].tolist())]
+    v2 = _bf_ln(xo, W["ln2_g"], W["ln2_b"])
+    f1 = [z * 0.5 * (1 + math.erf(z / math.sqrt(2))) for z in _bf_lin(v2, W["w_fc1"], W["b_fc1"])]
+    want = [p + r for p, r in zip(_bf_lin(f1, W["w_fc2"], W["b_fc2"]), xo)]
+    assert np.allclose(got[0], want, rtol=1e-10, atol=1e-10)
+    # the appended K codes are Q64 of fp16(K) from this step's projection input
+    c, m, s = q64.quantize(np.array(qkv[h:2 * h], np.float64).astype(np.float16))
+    assert np.array_equal(cache.t["k_codes"][0, :, pos].reshape(-1), c)
+
+
+def test_ln1_f16_prefill_rounds_projection_input():
+    """With the option on, the prefill's K rows are those of the projection
+    of fp16(LN1(x)); with it off, of LN1(x) itself."""
+    rng = np.random.default_rng(15)
+    for flag in (False, True):
+        cfg = tiny_cfg(ln1_f16=flag)
+        W = rand_layer(cfg, seed=16)
+        x = rng.standard_normal((1, 3, cfg.h))
+        _, K, _ = opt.layer_prefill(cfg, W, x)
+        for r in range(3):
+            u = _bf_ln(x[0, r].tolist(), W["ln1_g"], W["ln1_b"])
+            if flag:
+                u = [float(np.float16(v)) for v in u]
+            k = _bf_lin(u, W["w_qkv"][cfg.h:2 * cfg.h], W["b_qkv"][cfg.h:2 * cfg.h])
+            assert np.array_equal(K[0, r], np.array(k).astype(np.float16))
