@@ -190,6 +190,10 @@ def kernel_work(p: dict, kind: str, M: int, L_avg: float):
         byts = n * k * wb + M * k * 2 + M * n * 2 * (2 if res else 1) + n * 2
         return byts, 2.0 * M * n * k
     if kind == "attn_decode":
+        if p.get("topk_permille", 0) > 0:
+            # top-k sparse: every key, and the values of the kept keys only
+            kept = max(1.0, math.ceil(L_avg * p["topk_permille"] / 1000.0))
+            return M * a * (L_avg + kept) * kvb + 2 * M * h * 2, 2.0 * M * (L_avg + kept) * h
         return M * a * L_avg * 2 * kvb + 2 * M * h * 2, 4.0 * M * L_avg * h
     if kind == "attn_prefill":  # causal: half of the s x s score and value products
         return M * h * 2 * 4, 2.0 * M * L_avg * h
@@ -198,7 +202,8 @@ def kernel_work(p: dict, kind: str, M: int, L_avg: float):
     if kind == "layernorm":
         return M * h * 4 + 4 * h, 0.0
     if kind == "lm_head":
-        return p["vocab"] * h * 2 + M * h * 2 + M * p["vocab"] * 4, 2.0 * M * p["vocab"] * h
+        eb = 0.5 + 4 / 64 if p.get("embed_bits", 16) == 4 else 2.0
+        return p["vocab"] * h * eb + M * h * 2 + M * p["vocab"] * 4, 2.0 * M * p["vocab"] * h
     if kind == "argmax":
         return M * p["vocab"] * 4, 0.0
     if kind == "embed":
@@ -419,7 +424,7 @@ def run_reference(args, p):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": args.config, "global_batch": smp.b_o, "seq_len": p["s"],
+            "config": {"workload": workload_name(args), "global_batch": smp.b_o, "seq_len": p["s"],
                        "gen_tokens": p["n"], "note": "one layer per step, extrapolated"},
             "cpu_baseline": {"value": round(v, 4), "unit": "tokens/s", "cores": cpu_cores(),
                              "kind": "oracle",
@@ -431,6 +436,16 @@ def run_reference(args, p):
 
 
 METRIC = "decode tokens/s, OPT-30B-shape 4-bit W+KV; HBM GB/s & tensor util vs peak"
+
+
+def workload_name(args) -> str:
+    """The configuration's name, plus the variants that change the work."""
+    name = args.config
+    if args.embed_bits == 4:
+        name += "+embed4"
+    if args.topk:
+        name += f"+topk{args.topk}"
+    return name
 
 
 # ---------------------------------------------------------------------------
@@ -568,10 +583,13 @@ def run_flexq(args, p):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded splitmix64 draws; weights ~N(0,0.02) quantized to 4-bit)",
-            "config": {"workload": args.config, "layers": p["layers"], "h": p["h"],
+            "config": {"workload": workload_name(args), "layers": p["layers"], "h": p["h"],
                        "heads": p["heads"], "ffn": p["ffn"], "vocab": p["vocab"],
                        "global_batch": b * world, "gpu_batch": gbs, "seq_len": s,
                        "gen_tokens": n, "w_bits": p["w_bits"], "kv_bits": p["kv_bits"],
+                       "embed_bits": p.get("embed_bits", 16),
+                       "attn": (f"top-k sparse, {p['topk_permille'] / 10:g} % of keys"
+                                if p.get("topk_permille") else "dense"),
                        "parallelism": f"replicas x{world}",
                        "step": "decode phase: n-1 decode columns x all layers + LM head",
                        "l2": "no flush: inputs far larger than L2 (weights + KV per step)"},
@@ -614,10 +632,18 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-codec", action="store_true")
+    ap.add_argument("--embed-bits", type=int, default=16, choices=[16, 4],
+                    help="4: tied embedding / LM head stored group-wise 4-bit")
+    ap.add_argument("--topk", type=int, default=0,
+                    help="top-k sparse decode attention keeping ceil(L * TOPK / 1000) keys (100 = 10 %%)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
     p = dict(synth.CONFIGS[args.config])
+    if args.embed_bits != 16:
+        p["embed_bits"] = args.embed_bits
+    if args.topk:
+        p["topk_permille"] = args.topk
     if args.impl == "reference":
         run_reference(args, p)
     else:

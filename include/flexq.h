@@ -182,6 +182,9 @@ typedef struct {
   int w_bits;   /* 4 (packed tiled weights) or 16 (fp16 [N_out][K_in]) */
   int kv_bits;  /* 4 (group-wise codes) or 16 (fp16) */
   float ln_eps; /* LayerNorm epsilon (1e-5) */
+  int attn_topk_permille; /* 0: dense decode attention; 1..1000: top-k sparse
+                             decode attention keeping ceil(L * permille / 1000)
+                             keys (100 = the pages' top 10 %); 4-bit KV only */
 } flexq_config;
 
 /* One decoder layer's parameters (device pointers).  Linear weights [N_out]
@@ -232,6 +235,20 @@ flexq_status flexq_kv_append(const flexq_config* cfg, const flexq_kv* kv, const 
 flexq_status flexq_attention_decode(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev,
                                     int ldq, int b, int len, void* out_dev, int ldo, void* stream);
 
+/* Top-k sparse decode attention over a 4-bit cache ("FlexGen研究学术报告"
+ * section 三(C): only the top 10 % of the KV cache by attention value is
+ * loaded).  Per (sequence, head): scores s_t = q k_hat_t / sqrt(d) over all
+ * len slots, p = softmax(s) over all of them, T = the k slots with the
+ * largest scores (a lower slot wins a tie), out = sum_{t in T} p_t v_hat_t
+ * (full-softmax weights, not renormalised over T; k = len is dense
+ * attention).  K is read in full; V and its (min, scale) only for the 8-token
+ * blocks that hold a kept slot.  1 <= k <= len <= 16384.  idx_dev (may be
+ * NULL): int32 [b][heads][k], the kept slots in ascending order.  Scores,
+ * weights and sums are formed as in flexq_attention_decode. */
+flexq_status flexq_attention_decode_topk(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev, int ldq,
+                                         int b, int len, int k, void* out_dev, int ldo, int32_t* idx_dev,
+                                         void* stream);
+
 /* Causal prefill attention on fp16 Q/K/V: qkv_dev [b*s][ldqkv] with Q, K, V
  * at column offsets 0, h, 2h; out_dev [b*s][ldo]. */
 flexq_status flexq_attention_prefill(const flexq_config* cfg, const void* qkv_dev, int ldqkv,
@@ -257,7 +274,13 @@ flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* lay
 
 /* Decode of one layer for the token at position pos of b sequences: t_dev,
  * y_dev fp16 [b][h] (distinct).  Appends this token's K/V to slot pos, then
- * attends over slots 0..pos read back from the cache. */
+ * attends over slots 0..pos read back from the cache.  For b <= 256 the
+ * append happens inside the Q/K/V projection (its epilogue quantizes the
+ * K/V columns straight into the cache: the same codes flexq_kv_append gives
+ * those fp16 rows), LN2 runs inside the output projection (a cooperative
+ * launch whose CTAs normalise the finished rows after a grid-wide barrier),
+ * and decode attention over a 4-bit cache splits each head's cache over
+ * several CTAs when b * heads CTAs would not fill the GPU. */
 flexq_status flexq_layer_decode(const flexq_config* cfg, const flexq_layer* layer,
                                 const void* t_dev, void* y_dev, const flexq_kv* kv, int b,
                                 int pos, void* ws_dev, size_t ws_bytes, void* stream);
@@ -273,10 +296,17 @@ typedef struct {
   int max_pos;                /* rows of pos_embed */
   const flexq_layer* layer;   /* host array [layers] of device-pointer sets */
   const flexq_kv* kv;         /* host array [layers]; each b x max_len >= s+n */
-  const void* embed;          /* fp16 E [vocab][h]; also the tied LM head */
+  const void* embed;          /* word embedding E [vocab][h], also the tied LM head
+                                 ([WT] "内存占用分析"): fp16, or (embed_bits 4)
+                                 group-wise 4-bit in the tiled layout of
+                                 flexq_packed_weight_bytes(vocab, h), groups along
+                                 h; the lookups then read E's dequantized rows
+                                 fp16_rn(fp32(code * scale) + min) and the LM head
+                                 is the dequant-fused GEMM */
   const void* pos_embed;      /* fp16 P [max_pos][h] */
   const void* lnf_g;          /* final LayerNorm, fp16 [h] */
   const void* lnf_b;
+  int embed_bits;             /* 16 or 4: the format of embed */
 } flexq_model;
 
 typedef struct {
@@ -297,7 +327,15 @@ flexq_status flexq_generate_prefill(const flexq_model* model, const int32_t* pro
 /* The n-1 decode columns of flexq_generate alone: column j reads token
  * out_dev[i*n + j-1] at position s+j-1, appends its K/V to slot s+j-1 of every
  * layer and writes out_dev[i*n + j].  Needs the caches a prefill over the same
- * b sequences left (slots 0..s-1); re-running it rewrites slots s..s+n-2. */
+ * b sequences left (slots 0..s-1); re-running it rewrites slots s..s+n-2.
+ * With gpu_batch <= 256 each column is fused as in flexq_layer_decode, and
+ * further: the embedding kernel applies layer 0's LN1, and every layer's FC2
+ * kernel LayerNorms its output with the next layer's LN1 (the last layer's
+ * with the final LayerNorm), so a layer is five kernels (QKV + append,
+ * attention, output projection + LN, FC1 + GELU, FC2 + LN).  The split-tile
+ * counters in the workspace are zeroed once per call and every kernel leaves
+ * them zero; a kernel that gives up a bounded wait (FLEXQ_ERR_TIMEOUT) may
+ * leave them dirty, so results of the rest of that call are undefined. */
 flexq_status flexq_generate_decode(const flexq_model* model, int b, int s, int n, int gpu_batch,
                                    int32_t* out_dev, void* ws_dev, size_t ws_bytes, void* stream);
 
@@ -339,7 +377,10 @@ typedef enum {
  * launch is bracketed by two CUDA events on its stream (adds a little time;
  * one host thread at a time).  stop synchronises `stream` and writes, per
  * kind, the summed device milliseconds and the number of bracketed calls
- * (a linear layer's call also holds the memset of its split-tile counters). */
+ * (an unfused linear layer's call also holds the memset of its split-tile
+ * counters; a fused decode kernel counts under the kind of the linear layer
+ * or embedding it belongs to: the K/V append under QKV, LN2 under OUT_PROJ,
+ * the next LN1 or the final LayerNorm under FC2, layer 0's LN1 under EMBED). */
 flexq_status flexq_profile_start(void);
 flexq_status flexq_profile_stop(void* stream, float* total_ms /* [FLEXQ_K_COUNT] */,
                                 int* calls /* [FLEXQ_K_COUNT] */);

@@ -66,6 +66,8 @@ class Config:
     kv_bits: int = 4
     eps: float = 1e-5
     ln1_f16: bool = False
+    topk_permille: int = 0  # decode attention keeps the top ceil(L * permille / 1000) keys (0: dense)
+    embed_bits: int = 16    # 4: the tied embedding E is stored group-wise 4-bit (groups along h)
 
     @property
     def d(self) -> int:
@@ -75,7 +77,8 @@ class Config:
     def from_preset(p: dict, ln1_f16: bool = False) -> "Config":
         return Config(layers=p["layers"], h=p["h"], heads=p["heads"], ffn=p["ffn"],
                       vocab=p["vocab"], w_bits=p["w_bits"], kv_bits=p["kv_bits"],
-                      ln1_f16=ln1_f16)
+                      ln1_f16=ln1_f16, topk_permille=p.get("topk_permille", 0),
+                      embed_bits=p.get("embed_bits", 16))
 
 
 # ---------------------------------------------------------------------------
@@ -247,6 +250,42 @@ def attention_single(q, k, v):
     return np.einsum("bal,bald->bad", softmax(sc), v)
 
 
+def topk_count(L: int, permille: int) -> int:
+    """Keys kept by the top-k sparse attention: ceil(L * permille / 1000),
+    at least 1 and at most L ("FlexGen研究学术报告" section 三(C): only the
+    top 10 % of the cache by attention value is loaded; 10 % = 100 per mille)."""
+    return max(1, min(L, -(-L * permille // 1000)))
+
+
+def topk_select(scores, k):
+    """Indices of the k largest scores in ascending index order; among equal
+    scores the lower index is kept."""
+    order = sorted(range(len(scores)), key=lambda t: (-scores[t], t))
+    return sorted(order[:k])
+
+
+def attention_topk(q, k, v, kk):
+    """Top-k sparse decode attention.  q: [b, a, d]; k, v: [b, a, L, d];
+    kk keys kept per (sequence, head).  Scores and their softmax p are formed
+    over all L keys, exactly as dense attention; only the kk keys with the
+    largest scores contribute their values, with their softmax weights as
+    they are (no renormalisation over the kept keys): o = sum_{t in top-k}
+    p_t v_t.  With kk = L this is attention_single.  Returns (o [b, a, d],
+    selected indices [b, a, kk])."""
+    d = q.shape[-1]
+    sc = np.einsum("bad,bald->bal", q, k) / math.sqrt(d)
+    p = softmax(sc)
+    b, a, L = sc.shape
+    out = np.zeros((b, a, d))
+    sel = np.zeros((b, a, kk), dtype=np.int64)
+    for i in range(b):
+        for j in range(a):
+            idx = topk_select(sc[i, j].tolist(), kk)
+            sel[i, j] = idx
+            out[i, j] = p[i, j, idx] @ v[i, j, idx]
+    return out, sel
+
+
 # ---------------------------------------------------------------------------
 # Layer
 # ---------------------------------------------------------------------------
@@ -288,7 +327,11 @@ def layer_decode(cfg: Config, W: dict, t: np.ndarray, cache: KVCache, pos: int):
     cache.write("v", V.astype(np.float16)[:, None, :], pos)
     b = t.shape[0]
     q = Q.reshape(b, a, cfg.d)
-    o = attention_single(q, cache.read("k", pos + 1), cache.read("v", pos + 1)).reshape(b, h)
+    if cfg.topk_permille > 0:
+        kk = topk_count(pos + 1, cfg.topk_permille)
+        o = attention_topk(q, cache.read("k", pos + 1), cache.read("v", pos + 1), kk)[0].reshape(b, h)
+    else:
+        o = attention_single(q, cache.read("k", pos + 1), cache.read("v", pos + 1)).reshape(b, h)
     t_out = linear(o, W["w_o"], W["b_o"]) + t
     return _mlp(cfg, W, t_out)
 
@@ -307,9 +350,13 @@ class Model:
 
 
 def build_model(cfg: Config, seed: int, max_pos: int) -> Model:
+    """The model as it computes: effective layer weights, and the tied
+    embedding E as stored (its dequantized values when cfg.embed_bits == 4,
+    groups of 64 along h; the lookups and the LM head then both use them)."""
     layers = [effective_layer(cfg, raw_layer(cfg, seed, i)) for i in range(cfg.layers)]
     g = raw_globals(cfg, seed, max_pos)
-    return Model(cfg, layers, g["E"], g["P"], g["lnf_g"].astype(np.float64),
+    E = q64.roundtrip(g["E"]) if cfg.embed_bits == 4 else g["E"]
+    return Model(cfg, layers, E, g["P"], g["lnf_g"].astype(np.float64),
                  g["lnf_b"].astype(np.float64))
 
 

@@ -113,6 +113,8 @@ flexq_status check_config(const flexq_config* c) {
   FQ_CHECK(c->w_bits == 4 || c->w_bits == 16, "w_bits must be 4 or 16");
   FQ_CHECK(c->kv_bits == 4 || c->kv_bits == 16, "kv_bits must be 4 or 16");
   FQ_CHECK(c->ln_eps > 0.f, "ln_eps must be positive");
+  FQ_CHECK(c->attn_topk_permille >= 0 && c->attn_topk_permille <= 1000, "attn_topk_permille must be in 0..1000");
+  FQ_CHECK(c->attn_topk_permille == 0 || c->kv_bits == 4, "top-k sparse attention needs the 4-bit KV cache");
   return FLEXQ_OK;
 }
 
@@ -123,6 +125,9 @@ flexq_status check_kv(const flexq_config* c, const flexq_kv* kv, int b) {
   FQ_CHECK(kv->b >= b, "kv holds %d sequences, call needs %d", kv->b, b);
   FQ_CHECK(kv->max_len > 0, "kv->max_len must be positive");
   FQ_CHECK(aligned16(kv->k) && aligned16(kv->v), "KV buffers must be 16-byte aligned");
+  FQ_CHECK(c->kv_bits == 16 || ((reinterpret_cast<uintptr_t>(kv->k_meta) & 3) == 0 &&
+                                (reinterpret_cast<uintptr_t>(kv->v_meta) & 3) == 0),
+           "KV metadata must be 4-byte aligned");
   return FLEXQ_OK;
 }
 
@@ -159,13 +164,22 @@ KvView view_of(const flexq_config* c, const flexq_kv* kv, int seq0) {
 
 size_t align_up(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace layout of one layer step over M rows.
+// Workspace layout of one layer step over M rows.  ctr is a region that is
+// zeroed once per call and that the fused decode kernels leave zero: its
+// first 256 bytes hold the grid-barrier words, then the split-tile counters.
 struct LayerWs {
-  __half *u, *qkv, *xo, *g;
+  __half *u, *qkv, *xo, *g, *o, *v;
   float* acc;
   size_t acc_bytes;
+  float* attn_part;  // split decode attention partials
+  int* ctr;          // zeroed region: grid-barrier words | tile counters | attention counters
+  size_t ctr_bytes;
+  int* tile_ctr;
+  int* attn_ctr;
   size_t total;
 };
+
+constexpr size_t kSyncBytes = 256;
 
 LayerWs layer_ws_layout(const flexq_config* c, int M, uint8_t* base) {
   LayerWs w{};
@@ -180,20 +194,36 @@ LayerWs layer_ws_layout(const flexq_config* c, int M, uint8_t* base) {
   w.qkv = reinterpret_cast<__half*>(take(M * 3 * h * 2));
   w.xo = reinterpret_cast<__half*>(take(M * h * 2));
   w.g = reinterpret_cast<__half*>(take(M * f * 2));
-  size_t acc = 0;
-  acc = std::max(acc, linear_workspace_bytes(M, 3 * c->h, c->h, c->w_bits, 0));
-  acc = std::max(acc, linear_workspace_bytes(M, c->h, c->h, c->w_bits, 0));
-  acc = std::max(acc, linear_workspace_bytes(M, c->ffn, c->h, c->w_bits, 0));
-  acc = std::max(acc, linear_workspace_bytes(M, c->h, c->ffn, c->w_bits, 0));
+  w.o = reinterpret_cast<__half*>(take(M * h * 2));
+  w.v = reinterpret_cast<__half*>(take(M * h * 2));
+  const int shapes[4][2] = {{3 * c->h, c->h}, {c->h, c->h}, {c->ffn, c->h}, {c->h, c->ffn}};
+  size_t acc = 0, ctr = 0;
+  for (const auto& sh : shapes) {
+    acc = std::max(acc, linear_workspace_bytes(M, sh[0], sh[1], c->w_bits, 0));
+    ctr = std::max(ctr, linear_counter_bytes(M, sh[0], sh[1], c->w_bits, 0));
+  }
   w.acc_bytes = acc;
   w.acc = reinterpret_cast<float*>(take(acc));
+  const int d = c->h / c->heads;
+  w.attn_part = reinterpret_cast<float*>(take(attn_decode_partial_bytes(M, c->heads, d)));
+  const size_t attn_ctr = align_up(static_cast<size_t>(M) * c->heads * sizeof(int));
+  w.ctr_bytes = kSyncBytes + align_up(ctr) + attn_ctr;
+  w.ctr = reinterpret_cast<int*>(take(w.ctr_bytes));
+  w.tile_ctr = w.ctr ? w.ctr + kSyncBytes / sizeof(int) : nullptr;
+  w.attn_ctr = w.ctr ? w.tile_ctr + align_up(ctr) / sizeof(int) : nullptr;
   w.total = off;
   return w;
 }
 
+flexq_status zero_counters(const LayerWs& w, cudaStream_t s) {
+  FQ_CUDA(cudaMemsetAsync(w.ctr, 0, w.ctr_bytes, s), "zero split-tile counters");
+  return FLEXQ_OK;
+}
+
 flexq_status run_linear(const __half* x, int ldx, const void* w, int w_bits, int m, int n, int k,
                         const __half* bias, const __half* res, int ld_res, int epi, void* y, int ldy,
-                        void* ws, size_t ws_bytes, cudaStream_t s, const char* what) {
+                        void* ws, size_t ws_bytes, cudaStream_t s, const char* what,
+                        const KvFuse* kvf = nullptr, const LnFuse* lnf = nullptr, int* counters = nullptr) {
   LinearArgs a{};
   a.x = x;
   a.ldx = ldx;
@@ -208,7 +238,94 @@ flexq_status run_linear(const __half* x, int ldx, const void* w, int w_bits, int
   a.y = y;
   a.ldy = ldy;
   a.epi = epi;
+  a.kv = kvf;
+  a.ln = lnf;
+  a.counters = counters;
   FQ_CUDA(launch_linear(a, ws, ws_bytes, s), what);
+  return FLEXQ_OK;
+}
+
+// Decode attention of a layer step: dense, or top-k sparse when the config
+// asks for it.
+cudaError_t decode_attention(const flexq_config* c, const __half* q, int ldq, const KvView& kvv, int b, int len,
+                             __half* out, int ldo, float* part, int* ctr, cudaStream_t s) {
+  const int d = c->h / c->heads;
+  if (c->attn_topk_permille > 0)
+    return launch_attn_topk(q, ldq, kvv, b, c->heads, d, len, topk_count(len, c->attn_topk_permille), out, ldo,
+                            nullptr, s);
+  return launch_attn_decode(q, ldq, kvv, b, c->heads, d, c->kv_bits, len, out, ldo, part, ctr, s);
+}
+
+// The fused decode step takes at most one token tile of sequences.
+bool decode_fusable(int b) { return b >= 1 && b <= kFuseMaxRows; }
+
+// Decode step of one layer for b sequences, fused ([WT] "P/D阶段计算",
+// decoding phase): u_in = LN1(t) computed by the caller (the previous
+// layer's FC2 or the embedding); the QKV projection appends this token's K/V
+// to cache slot pos in its epilogue; attention reads slots 0..pos; the
+// output projection adds the residual and LayerNorms its rows (LN2) after a
+// grid barrier; FC1 + GELU; FC2 adds the residual and, when ln_next_g is
+// set, LayerNorms its rows into u_out (the next layer's LN1 or the final
+// LN).  w.ctr must be zero (it is left zero).
+flexq_status decode_fused(const flexq_config* c, const flexq_layer* L, const __half* t, const __half* u_in,
+                          __half* y, __half* u_out, const void* ln_next_g, const void* ln_next_b,
+                          const flexq_kv* kv, int seq0, int b, int pos, const LayerWs& w, cudaStream_t s) {
+  const int h = c->h, f = c->ffn, d = h / c->heads;
+  const KvView kvv = view_of(c, kv, seq0);
+  int* tile_ctr = w.tile_ctr;
+  KvFuse kf{};
+  kf.k_codes = static_cast<uint8_t*>(kvv.k);
+  kf.v_words = static_cast<uint32_t*>(kvv.v);
+  kf.k_meta = static_cast<__half2*>(kvv.k_meta);
+  kf.v_meta = static_cast<__half2*>(kvv.v_meta);
+  kf.h = h;
+  kf.heads = c->heads;
+  kf.d = d;
+  kf.max_len = kvv.max_len;
+  kf.pos = pos;
+  kf.bits = c->kv_bits;
+  {
+    ProfScope ps(FLEXQ_K_QKV, s);
+    FQ_TRY(run_linear(u_in, h, L->w_qkv, c->w_bits, b, 3 * h, h, static_cast<const __half*>(L->b_qkv), nullptr, 0,
+                      EPI_BIAS, w.qkv, 3 * h, w.acc, w.acc_bytes, s, "QKV projection with KV append", &kf, nullptr,
+                      tile_ctr));
+  }
+  {
+    ProfScope ps(FLEXQ_K_ATTN_DECODE, s);
+    FQ_CUDA(decode_attention(c, w.qkv, 3 * h, kvv, b, pos + 1, w.o, h, w.attn_part, w.attn_ctr, s),
+            "decode attention");
+  }
+  LnFuse ln2{};
+  ln2.g = static_cast<const __half*>(L->ln2_g);
+  ln2.b = static_cast<const __half*>(L->ln2_b);
+  ln2.y = w.v;
+  ln2.ldy = h;
+  ln2.eps = c->ln_eps;
+  ln2.sync = w.ctr;
+  {
+    ProfScope ps(FLEXQ_K_OUT_PROJ, s);
+    FQ_TRY(run_linear(w.o, h, L->w_o, c->w_bits, b, h, h, static_cast<const __half*>(L->b_o), t, h,
+                      EPI_BIAS | EPI_RESIDUAL, w.xo, h, w.acc, w.acc_bytes, s, "output projection with LN2",
+                      nullptr, &ln2, tile_ctr));
+  }
+  {
+    ProfScope ps(FLEXQ_K_FC1, s);
+    FQ_TRY(run_linear(w.v, h, L->w_fc1, c->w_bits, b, f, h, static_cast<const __half*>(L->b_fc1), nullptr, 0,
+                      EPI_BIAS | EPI_GELU, w.g, f, w.acc, w.acc_bytes, s, "FC1", nullptr, nullptr, tile_ctr));
+  }
+  LnFuse lnn{};
+  lnn.g = static_cast<const __half*>(ln_next_g);
+  lnn.b = static_cast<const __half*>(ln_next_b);
+  lnn.y = u_out;
+  lnn.ldy = h;
+  lnn.eps = c->ln_eps;
+  lnn.sync = w.ctr;
+  {
+    ProfScope ps(FLEXQ_K_FC2, s);
+    FQ_TRY(run_linear(w.g, f, L->w_fc2, c->w_bits, b, h, f, static_cast<const __half*>(L->b_fc2), w.xo, h,
+                      EPI_BIAS | EPI_RESIDUAL, y, h, w.acc, w.acc_bytes, s, "FC2",
+                      nullptr, ln_next_g != nullptr ? &lnn : nullptr, tile_ctr));
+  }
   return FLEXQ_OK;
 }
 
@@ -239,8 +356,7 @@ flexq_status layer_step(const flexq_config* c, const flexq_layer* L, const __hal
     FQ_CUDA(launch_attn_prefill(w.qkv, 3 * h, b, ntok, c->heads, d, w.u, h, s), "prefill attention");
   } else {
     ProfScope ps(FLEXQ_K_ATTN_DECODE, s);
-    FQ_CUDA(launch_attn_decode(w.qkv, 3 * h, kvv, b, c->heads, d, c->kv_bits, pos + 1, w.u, h, s),
-            "decode attention");
+    FQ_CUDA(decode_attention(c, w.qkv, 3 * h, kvv, b, pos + 1, w.u, h, nullptr, nullptr, s), "decode attention");
   }
   {
     ProfScope ps(FLEXQ_K_OUT_PROJ, s);
@@ -302,7 +418,7 @@ extern "C" {
 
 const char* flexq_last_error(void) { return g_last_error.c_str(); }
 
-int flexq_version(void) { return 100; }
+int flexq_version(void) { return 101; }
 
 flexq_status flexq_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns = ns == 0 ? 2000000000ull : ns;
@@ -496,9 +612,26 @@ flexq_status flexq_attention_decode(const flexq_config* cfg, const flexq_kv* kv,
   FQ_CHECK(q_dev && out_dev, "NULL pointer");
   FQ_CHECK(ldq >= cfg->h && ldo >= cfg->h && ldq % 8 == 0 && ldo % 8 == 0, "bad row strides");
   FQ_CUDA(launch_attn_decode(static_cast<const __half*>(q_dev), ldq, view_of(cfg, kv, 0), b, cfg->heads,
-                             cfg->h / cfg->heads, cfg->kv_bits, len, static_cast<__half*>(out_dev), ldo,
-                             as_stream(stream)),
+                             cfg->h / cfg->heads, cfg->kv_bits, len, static_cast<__half*>(out_dev), ldo, nullptr,
+                             nullptr, as_stream(stream)),
           "decode attention");
+  return FLEXQ_OK;
+}
+
+flexq_status flexq_attention_decode_topk(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev, int ldq,
+                                         int b, int len, int k, void* out_dev, int ldo, int32_t* idx_dev,
+                                         void* stream) {
+  FQ_TRY(check_config(cfg));
+  FQ_CHECK(cfg->kv_bits == 4, "top-k sparse attention reads the 4-bit cache");
+  FQ_TRY(check_kv(cfg, kv, b));
+  FQ_CHECK(len >= 1 && len <= kv->max_len && len <= 16384, "len must be in 1..min(max_len, 16384)");
+  FQ_CHECK(k >= 1 && k <= len, "k must be in 1..len");
+  if (b == 0) return FLEXQ_OK;
+  FQ_CHECK(q_dev && out_dev, "NULL pointer");
+  FQ_CHECK(ldq >= cfg->h && ldo >= cfg->h && ldq % 8 == 0 && ldo % 8 == 0, "bad row strides");
+  FQ_CUDA(launch_attn_topk(static_cast<const __half*>(q_dev), ldq, view_of(cfg, kv, 0), b, cfg->heads,
+                           cfg->h / cfg->heads, len, k, static_cast<__half*>(out_dev), ldo, idx_dev, as_stream(stream)),
+          "top-k decode attention");
   return FLEXQ_OK;
 }
 
@@ -539,8 +672,19 @@ static flexq_status layer_common(const flexq_config* cfg, const flexq_layer* lay
     return fail(FLEXQ_ERR_WORKSPACE, "layer needs %zu workspace bytes, got %zu", probe.total, ws_bytes);
   FQ_CHECK(aligned16(ws), "workspace must be 16-byte aligned");
   const LayerWs w = layer_ws_layout(cfg, M, static_cast<uint8_t*>(ws));
-  return layer_step(cfg, layer, static_cast<const __half*>(x), static_cast<__half*>(y), kv, 0, b, ntok, pos,
-                    prefill, w, as_stream(stream));
+  cudaStream_t st = as_stream(stream);
+  if (prefill || !decode_fusable(b))
+    return layer_step(cfg, layer, static_cast<const __half*>(x), static_cast<__half*>(y), kv, 0, b, ntok, pos,
+                      prefill, w, st);
+  FQ_TRY(zero_counters(w, st));
+  {
+    ProfScope ps(FLEXQ_K_LAYERNORM, st);
+    FQ_CUDA(launch_layernorm(static_cast<const __half*>(x), cfg->h, static_cast<const __half*>(layer->ln1_g),
+                             static_cast<const __half*>(layer->ln1_b), w.u, cfg->h, b, cfg->h, cfg->ln_eps, st),
+            "LayerNorm 1");
+  }
+  return decode_fused(cfg, layer, static_cast<const __half*>(x), w.u, static_cast<__half*>(y), nullptr, nullptr,
+                      nullptr, kv, 0, b, pos, w, st);
 }
 
 flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* layer, const void* x_dev, void* y_dev,
@@ -588,7 +732,7 @@ GenWs gen_ws_layout(const flexq_model* m, int b, int s, int gbs, uint8_t* base) 
   w.layer_bytes =
       std::max(layer_ws_layout(&m->cfg, gbs * s, nullptr).total, layer_ws_layout(&m->cfg, gbs, nullptr).total);
   w.layer = take(w.layer_bytes);
-  w.head_acc_bytes = linear_workspace_bytes(b, m->vocab, m->cfg.h, 16, 0);
+  w.head_acc_bytes = linear_workspace_bytes(b, m->vocab, m->cfg.h, m->embed_bits == 4 ? 4 : 16, 0);
   w.head_acc = reinterpret_cast<float*>(take(w.head_acc_bytes));
   w.total = off;
   return w;
@@ -600,6 +744,9 @@ flexq_status check_model(const flexq_model* m) {
   FQ_CHECK(m->layers > 0 && m->layer && m->kv, "model needs layers, layer and kv arrays");
   FQ_CHECK(m->vocab > 0 && m->max_pos > 0, "vocab and max_pos must be positive");
   FQ_CHECK(m->embed && m->pos_embed && m->lnf_g && m->lnf_b, "model embedding/final LN pointer is NULL");
+  FQ_CHECK(m->embed_bits == 16 || m->embed_bits == 4, "embed_bits must be 16 or 4");
+  FQ_CHECK(aligned16(m->embed) && aligned16(m->pos_embed) && aligned16(m->lnf_g) && aligned16(m->lnf_b),
+           "embedding and final LayerNorm tensors must be 16-byte aligned");
   for (int i = 0; i < m->layers; ++i) FQ_TRY(check_layer(&m->cfg, &m->layer[i]));
   return FLEXQ_OK;
 }
@@ -625,10 +772,12 @@ flexq_status check_generation(const flexq_model* model, int b, int s, int n, int
   return FLEXQ_OK;
 }
 
+// Final LayerNorm (unless the rows arrive normalised in w.tn), tied LM head
+// and greedy choice.
 flexq_status lm_head(const flexq_model* m, const __half* x_last, int ldx, int b, const GenWs& w, int32_t* out,
-                     int ld_out, cudaStream_t s) {
+                     int ld_out, cudaStream_t s, bool normalised = false) {
   const int h = m->cfg.h;
-  {
+  if (!normalised) {
     ProfScope ps(FLEXQ_K_LAYERNORM, s);
     FQ_CUDA(launch_layernorm(x_last, ldx, static_cast<const __half*>(m->lnf_g),
                              static_cast<const __half*>(m->lnf_b), w.tn, h, b, h, m->cfg.ln_eps, s),
@@ -636,7 +785,8 @@ flexq_status lm_head(const flexq_model* m, const __half* x_last, int ldx, int b,
   }
   {
     ProfScope ps(FLEXQ_K_LM_HEAD, s);
-    FQ_TRY(run_linear(w.tn, h, m->embed, 16, b, m->vocab, h, nullptr, nullptr, 0, EPI_F32_OUT, w.logits, m->vocab,
+    FQ_TRY(run_linear(w.tn, h, m->embed, m->embed_bits, b, m->vocab, h, nullptr, nullptr, 0, EPI_F32_OUT, w.logits,
+                      m->vocab,
                       w.head_acc, w.head_acc_bytes, s, "LM head"));
   }
   ProfScope ps(FLEXQ_K_ARGMAX, s);
@@ -652,7 +802,7 @@ flexq_status prefill_column(const flexq_model* model, const int32_t* prompt_dev,
   const int h = c->h, nb = b / gpu_batch;
   {
     ProfScope ps(FLEXQ_K_EMBED, st);
-    FQ_CUDA(launch_embed(prompt_dev, s, b, s, static_cast<const __half*>(model->embed), model->vocab,
+    FQ_CUDA(launch_embed(prompt_dev, s, b, s, model->embed, model->embed_bits, model->vocab,
                          static_cast<const __half*>(model->pos_embed), 0, h, w.x, st),
             "embedding");
   }
@@ -676,11 +826,43 @@ flexq_status decode_columns(const flexq_model* model, int b, int s, int n, int g
   const flexq_config* c = &model->cfg;
   const int h = c->h, nb = b / gpu_batch;
   const LayerWs lw = layer_ws_layout(c, gpu_batch, w.layer);
+  if (decode_fusable(gpu_batch)) {
+    // Fused columns: the embedding applies layer 0's LN1; each layer's FC2
+    // LayerNorms its output with the next layer's LN1 (the last layer's with
+    // the final LN) into w.tn, which the next QKV projection (or the LM
+    // head) reads.  The counters are zeroed once for all columns.
+    FQ_TRY(zero_counters(lw, st));
+    for (int j = 1; j < n; ++j) {
+      const int pos = s + j - 1;
+      {
+        ProfScope ps(FLEXQ_K_EMBED, st);
+        FQ_CUDA(launch_embed_ln(out_dev + (j - 1), n, b, model->embed, model->embed_bits, model->vocab,
+                                static_cast<const __half*>(model->pos_embed), pos, h, w.t,
+                                static_cast<const __half*>(model->layer[0].ln1_g),
+                                static_cast<const __half*>(model->layer[0].ln1_b), c->ln_eps, w.tn, st),
+                "embedding with LN1");
+      }
+      __half *t = w.t, *t2 = w.t2;
+      for (int l = 0; l < model->layers; ++l) {
+        const bool last = l + 1 == model->layers;
+        const void* g = last ? model->lnf_g : model->layer[l + 1].ln1_g;
+        const void* bb = last ? model->lnf_b : model->layer[l + 1].ln1_b;
+        for (int k = 0; k < nb; ++k) {
+          const size_t off = static_cast<size_t>(k) * gpu_batch * h;
+          FQ_TRY(decode_fused(c, &model->layer[l], t + off, w.tn + off, t2 + off, w.tn + off, g, bb, &model->kv[l],
+                              k * gpu_batch, gpu_batch, pos, lw, st));
+        }
+        std::swap(t, t2);
+      }
+      FQ_TRY(lm_head(model, w.tn, h, b, w, out_dev + j, n, st, true));
+    }
+    return FLEXQ_OK;
+  }
   for (int j = 1; j < n; ++j) {
     const int pos = s + j - 1;
     {
       ProfScope ps(FLEXQ_K_EMBED, st);
-      FQ_CUDA(launch_embed(out_dev + (j - 1), n, b, 1, static_cast<const __half*>(model->embed), model->vocab,
+      FQ_CUDA(launch_embed(out_dev + (j - 1), n, b, 1, model->embed, model->embed_bits, model->vocab,
                            static_cast<const __half*>(model->pos_embed), pos, h, w.t, st),
               "embedding");
     }

@@ -46,6 +46,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "quant_common.cuh"
 
 namespace flexq {
 namespace {
@@ -60,6 +61,7 @@ constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
 constexpr int kMaxBarriers = 56;     // mbarriers fit in the first 448 bytes of that region
 constexpr int kEpiStageBytes = 4 * 16 * 33 * 4;  // per epilogue warp: 16 tokens x 33 floats
+constexpr int kKvStageBytes = 16 * 128 * 2;      // fp16 K/V rows of 16 tokens x 128 features
 constexpr int kMaxLoadStages = 16;
 constexpr int kMinItersPerCta = 8;
 constexpr int kMaxContrib = 64;
@@ -99,6 +101,10 @@ struct GemmParams {
   int* counters;    // [tiles][2]: contributors arrived, partials published
   uint64_t wait_ns;
   uint32_t* err;
+  int kv_on;        // decode QKV: K/V tiles go to the 4-bit cache
+  KvFuse kv;
+  int ln_on;        // decode out-proj / FC2: LayerNorm of the rows after a grid barrier
+  LnFuse ln;
 };
 
 struct Seg {
@@ -300,6 +306,7 @@ struct Ctl {
   volatile int* fin_me;
   int* fin_slots;  // [kMaxContrib]
   float* stage;    // [4][16][33]
+  __half* kvst;    // [16][128] fp16 K/V rows of the chunk being quantized
 };
 
 __device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
@@ -313,7 +320,68 @@ __device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
   c.fin_me = c.abort_flag + 3;
   c.fin_slots = reinterpret_cast<int*>(region + kBarrierBytes / 2);
   c.stage = reinterpret_cast<float*>(region + kBarrierBytes);
+  c.kvst = reinterpret_cast<__half*>(region + kBarrierBytes + kEpiStageBytes);
   return c;
+}
+
+// Quantizes the staged fp16 K/V rows of one 16-token chunk into the cache:
+// thread et (< 64, two whole warps) and its neighbour et ^ 1 own one
+// 64-feature group of one token, exactly as the standalone append kernels
+// split a row ("FlexGen研究学术报告" section 三(C): groups of 64 along the
+// head dimension, fp16 min/scale).  K: canonical codes of slot pos; V: the
+// token's nibble in each token-interleaved word (one writer per word, since
+// a decode step appends a single token per sequence).
+__device__ __forceinline__ void kv_quantize_chunk(const GemmParams& p, const __half* kvst, int tokbase,
+                                                  int n_tile, int et) {
+  const int jq = et >> 2, gq = (et >> 1) & 1, half_id = et & 1;
+  const uint4* src = reinterpret_cast<const uint4*>(kvst + jq * 128 + gq * 64 + half_id * 32);
+  float v[32];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint4 w = src[u];
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(u32_as_h2(ww[e]));
+      v[8 * u + 2 * e] = f.x;
+      v[8 * u + 2 * e + 1] = f.y;
+    }
+  }
+  uint32_t q[32];
+  __half m16, s16;
+  q64_lane_pair(v, q, m16, s16);
+  const int tok = tokbase + jq;
+  if (tok >= p.m) return;
+  const KvFuse& kv = p.kv;
+  const int col = n_tile * 128 + gq * 64;
+  const bool is_v = col >= 2 * kv.h;
+  const int cc = col - (is_v ? 2 * kv.h : kv.h);
+  const int j = cc / kv.d, gd = (cc % kv.d) / 64;
+  const size_t hr = static_cast<size_t>(tok) * kv.heads + j;
+  const size_t slot = hr * kv.max_len + kv.pos;
+  if (!is_v) {
+    const uint4 out = make_uint4(pack_canonical(q), pack_canonical(q + 8), pack_canonical(q + 16),
+                                 pack_canonical(q + 24));
+    *reinterpret_cast<uint4*>(kv.k_codes + slot * (kv.d / 2) + gd * 32 + half_id * 16) = out;
+    if (half_id == 0) kv.k_meta[slot * (kv.d / 64) + gd] = __halves2half2(m16, s16);
+  } else {
+    uint4* w4 = reinterpret_cast<uint4*>(kv.v_words + (hr * (kv_pad_len(kv.max_len) / 8) + kv.pos / 8) * kv.d +
+                                         gd * 64 + half_id * 32);
+    const int sh = 4 * (kv.pos & 7);
+    const uint32_t clear = ~(0xFu << sh);
+    uint4 cur[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cur[u] = w4[u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cur[u].x = (cur[u].x & clear) | (q[4 * u] << sh);
+      cur[u].y = (cur[u].y & clear) | (q[4 * u + 1] << sh);
+      cur[u].z = (cur[u].z & clear) | (q[4 * u + 2] << sh);
+      cur[u].w = (cur[u].w & clear) | (q[4 * u + 3] << sh);
+      w4[u] = cur[u];
+    }
+    if (half_id == 0) kv.v_meta[slot * (kv.d / 64) + gd] = __halves2half2(m16, s16);
+  }
 }
 
 // Bounded wait until a global counter reaches `target` (the other
@@ -359,6 +427,8 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
     const uint32_t tbase =
         tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + (static_cast<uint32_t>(qd * 32) << 16);
     const int f_out = n_tile * 128 + qd * 32 + hf * 16;  // features this lane finishes
+    // decode QKV with the cache fused: the K and V tiles are quantized, not stored
+    const bool kv_tile = p.kv_on && n_tile * 128 >= p.kv.h;
     // Split tile: count in; the last to arrive finishes the tile.
     int ns = 1, me = 0;
     if (!g.full) {
@@ -469,7 +539,37 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = v[j];
       __syncwarp();
       const int tok = tok0 + c0 + jt;
-      if (tok < p.m && f_out < p.n) {
+      if (kv_tile) {
+        // the chunk's fp16 rows (+ bias, the values the cache receives)
+        uint32_t packed[8];
+#pragma unroll
+        for (int u = 0; u < 16; u += 2)
+          packed[u / 2] = h2_as_u32(__floats2half2_rn(stg[jt * 33 + hf * 16 + u] + bv[u],
+                                                      stg[jt * 33 + hf * 16 + u + 1] + bv[u + 1]));
+        if (p.kv.bits == 16) {
+          // fp16 cache: this lane's 16 features of its token go to slot pos
+          if (tok < p.m) {
+            const bool is_v = f_out >= 2 * p.kv.h;
+            const int cc = f_out - (is_v ? 2 * p.kv.h : p.kv.h);
+            __half* base = reinterpret_cast<__half*>(is_v ? static_cast<void*>(p.kv.v_words)
+                                                          : static_cast<void*>(p.kv.k_codes));
+            uint4* dst = reinterpret_cast<uint4*>(
+                base + ((static_cast<size_t>(tok) * p.kv.heads + cc / p.kv.d) * p.kv.max_len + p.kv.pos) * p.kv.d +
+                cc % p.kv.d);
+            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          }
+        } else {
+          // 4-bit cache: stage in shared memory; two warps then quantize
+          // whole 64-feature groups
+          uint4* dst = reinterpret_cast<uint4*>(c.kvst + jt * 128 + qd * 32 + hf * 16);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+          epi_bar();
+          if (et < 64) kv_quantize_chunk(p, c.kvst, tok0 + c0, n_tile, et);
+          epi_bar();
+        }
+      } else if (tok < p.m && f_out < p.n) {
         float o[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) o[u] = stg[jt * 33 + hf * 16 + u];
@@ -477,8 +577,129 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       }
       __syncwarp();
     }
+    // A split tile's counters go back to zero once it is finished (every
+    // contributor has counted in and published), so a sequence of launches
+    // needs them zeroed only once.
+    if (!g.full && et == 0) {
+      p.counters[2 * g.tile] = 0;
+      p.counters[2 * g.tile + 1] = 0;
+    }
     tc_fence_before();
     mbar_arrive(&c.acce[buf]);
+  }
+}
+
+// Grid-wide barrier of a cooperative launch, entered by one thread per CTA
+// after its CTA's stores are complete.  sync[0] counts arrivals, sync[1] is
+// the generation: the last arrival resets the count and advances the
+// generation, the others wait (bounded) for the generation to move.  Both
+// words return to their entry values' pattern (count 0), so one zeroing
+// serves every later launch.
+__device__ __forceinline__ bool grid_sync(int* sync, int nblocks, uint64_t limit_ns) {
+  int g0;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(g0) : "l"(sync + 1) : "memory");
+  __threadfence();
+  const int old = atomicAdd(sync, 1);
+  if (old == nblocks - 1) {
+    atomicExch(sync, 0);
+    __threadfence();
+    atomicAdd(sync + 1, 1);
+    return true;
+  }
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    int g;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(g) : "l"(sync + 1) : "memory");
+    if (g != g0) break;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+    __nanosleep(32);
+  }
+  __threadfence();
+  return true;
+}
+
+__device__ __forceinline__ float block_sum_all(float v, float* red) {
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane_id() == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = 0.f;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) r += red[w];
+  return r;
+}
+
+// LayerNorm phase of the fused out-proj / FC2 (after every CTA's tiles are
+// stored): rows blockIdx.x, blockIdx.x + grid, ... of the fp16 output are
+// normalised by all threads of the CTA with fp32 statistics (biased
+// variance, two passes over registers) and written to p.ln.y.
+constexpr int kLnVec = 4;  // 16-byte vectors per thread: h <= 448 * 4 * 8
+__device__ void ln_phase(const GemmParams& p, const Ctl& c) {
+  __syncthreads();
+  volatile int* ok_flag = c.last_flag;
+  if (threadIdx.x == 0) {
+    const bool mine = *c.abort_flag == 0;
+    const bool met = grid_sync(p.ln.sync, gridDim.x, drain_ns(p.wait_ns));
+    if (!met) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
+    *ok_flag = mine && met;
+  }
+  __syncthreads();
+  if (!*ok_flag) return;
+  float* red = c.stage;
+  const int nvec = p.n / 8;
+  for (int r = blockIdx.x; r < p.m; r += gridDim.x) {
+    const uint4* xr = reinterpret_cast<const uint4*>(p.y + static_cast<size_t>(r) * p.ldy);
+    float v[kLnVec][8];
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kLnVec; ++i) {
+      const int vi = threadIdx.x + i * kThreads;
+      if (vi < nvec) {
+        const uint4 u = __ldcg(xr + vi);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(u32_as_h2(w[e]));
+          v[i][2 * e] = f.x;
+          v[i][2 * e + 1] = f.y;
+          sum += f.x + f.y;
+        }
+      }
+    }
+    const float mean = block_sum_all(sum, red) / static_cast<float>(p.n);
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < kLnVec; ++i) {
+      if (threadIdx.x + i * kThreads < nvec) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float dl = v[i][e] - mean;
+          sq += dl * dl;
+        }
+      }
+    }
+    const float var = block_sum_all(sq, red + 16) / static_cast<float>(p.n);
+    const float rstd = 1.0f / sqrtf(var + p.ln.eps);
+    uint4* yr = reinterpret_cast<uint4*>(p.ln.y + static_cast<size_t>(r) * p.ln.ldy);
+#pragma unroll
+    for (int i = 0; i < kLnVec; ++i) {
+      const int vi = threadIdx.x + i * kThreads;
+      if (vi < nvec) {
+        const uint4 gu = reinterpret_cast<const uint4*>(p.ln.g)[vi];
+        const uint4 bu = reinterpret_cast<const uint4*>(p.ln.b)[vi];
+        const uint32_t gw[4] = {gu.x, gu.y, gu.z, gu.w};
+        const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 gf = __half22float2(u32_as_h2(gw[e]));
+          const float2 bf = __half22float2(u32_as_h2(bw[e]));
+          o[e] = h2_as_u32(__floats2half2_rn((v[i][2 * e] - mean) * rstd * gf.x + bf.x,
+                                             (v[i][2 * e + 1] - mean) * rstd * gf.y + bf.y));
+        }
+        yr[vi] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
   }
 }
 
@@ -700,6 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     epilogue_role(p, c, tmem_base, warp, lane);
   }
   teardown(p, c, tmem_base, warp);
+  if (p.ln_on) ln_phase(p, c);
 }
 
 // ---------------------------------------------------------------------------
@@ -843,7 +1065,7 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.partial_bytes = static_cast<size_t>(2) * s.grid * tile_bytes;
   }
   if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * 2 * sizeof(int);
-  const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
+  const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes - kKvStageBytes;
   const int b_bytes = P.tok_tile * 128;
   int a_slot = 0;
   {
@@ -862,7 +1084,7 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   }
   P.load_stages = min(kMaxLoadStages, (budget - P.a_stages * a_slot) / static_cast<int>(P.load_stage_bytes));
   P.smem = static_cast<size_t>(P.a_stages) * a_slot + static_cast<size_t>(P.load_stages) * P.load_stage_bytes +
-           1024 + kBarrierBytes + kEpiStageBytes;
+           1024 + kBarrierBytes + kEpiStageBytes + kKvStageBytes;
   return P;
 }
 
@@ -878,12 +1100,29 @@ cudaError_t configure_once() {
   return status;
 }
 
+// A fused LayerNorm needs every CTA resident at once (grid barrier), so that
+// variant is a cooperative launch; the grid never exceeds one CTA per SM.
 template <bool kW4, int KS>
 cudaError_t launch_general(const Plan& P, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                            cudaStream_t s) {
   const cudaError_t e = configure_once<gemm_tc_kernel<kW4, KS>>();
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<kW4, KS><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
+  if (!p.ln_on) {
+    gemm_tc_kernel<kW4, KS><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
+    return launched();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.sc.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = P.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<kW4, KS>, tx, tw, p);
+  if (le != cudaSuccess) return le;
   return launched();
 }
 
@@ -893,6 +1132,14 @@ size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits)
   const Plan P = make_plan(m, n, k, w_bits, force_splits, 0);
   if (P.partial_bytes == 0) return 0;
   return align256(P.partial_bytes) + align256(P.counter_bytes);
+}
+
+size_t linear_counter_bytes(int m, int n, int k, int w_bits, int force_splits) {
+  return make_plan(m, n, k, w_bits, force_splits, 0).counter_bytes;
+}
+
+size_t linear_partial_bytes(int m, int n, int k, int w_bits, int force_splits) {
+  return make_plan(m, n, k, w_bits, force_splits, 0).partial_bytes;
 }
 
 cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaStream_t s) {
@@ -939,12 +1186,33 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
     p.ldy = a.ldy;
   }
   if (P.partial_bytes > 0) {
-    const size_t need = align256(P.partial_bytes) + align256(P.counter_bytes);
-    if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
-    p.partials = static_cast<float*>(ws);
-    p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + align256(P.partial_bytes));
-    const cudaError_t e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
-    if (e != cudaSuccess) return e;
+    if (a.counters != nullptr) {
+      if (ws == nullptr || ws_bytes < P.partial_bytes) return cudaErrorInvalidValue;
+      p.partials = static_cast<float*>(ws);
+      p.counters = a.counters;
+    } else {
+      const size_t need = align256(P.partial_bytes) + align256(P.counter_bytes);
+      if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
+      p.partials = static_cast<float*>(ws);
+      p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + align256(P.partial_bytes));
+      const cudaError_t e = cudaMemsetAsync(p.counters, 0, P.counter_bytes, s);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  if (a.kv != nullptr) {
+    // whole 64-feature groups of one head per K/V tile; one token tile
+    if (a.m > kFuseMaxRows || P.tok_tiles != 1 || a.n != 3 * a.kv->h || a.kv->h % 128 != 0 ||
+        (a.epi & ~EPI_BIAS) != 0 || (a.kv->bits != 4 && a.kv->bits != 16))
+      return cudaErrorInvalidValue;
+    p.kv_on = 1;
+    p.kv = *a.kv;
+  }
+  if (a.ln != nullptr) {
+    if (a.m > kFuseMaxRows || (a.epi & EPI_F32_OUT) || a.n % 8 != 0 || a.n > kThreads * 8 * 4 ||
+        a.ln->sync == nullptr || P.sc.grid > runtime().num_sms)
+      return cudaErrorInvalidValue;
+    p.ln_on = 1;
+    p.ln = *a.ln;
   }
   if (w4 && P.ks == 2) return launch_general<true, 2>(P, tx, tw, p, s);
   if (w4) return launch_general<true, 1>(P, tx, tw, p, s);

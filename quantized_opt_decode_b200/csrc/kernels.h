@@ -66,6 +66,10 @@ cudaError_t launch_kv_append(const __half* k_src, const __half* v_src, int ld_sr
 // LayerNorm over rows of width h (fp16 in/out, fp32 statistics)
 cudaError_t launch_layernorm(const __half* x, int ldx, const __half* g, const __half* bta,
                              __half* y, int ldy, int rows, int h, float eps, cudaStream_t s);
+// Bytes of the split-tile counters a linear layer of this shape uses (0 when
+// it splits no tile), and of its partial tiles alone.
+size_t linear_counter_bytes(int m, int n, int k, int w_bits, int force_splits);
+size_t linear_partial_bytes(int m, int n, int k, int w_bits, int force_splits);
 
 // GEMM: Y[m][n] = epilogue(X[m][k] . W[n][k]^T)
 enum Epilogue : int {
@@ -73,6 +77,29 @@ enum Epilogue : int {
   EPI_GELU = 2,       // GELU (exact erf form) after the bias
   EPI_RESIDUAL = 4,   // + residual[m][n] last
   EPI_F32_OUT = 8,    // write fp32 (no bias/act/residual allowed)
+};
+// Decode-step fusions of a linear layer (one token per sequence, m rows):
+// KvFuse makes the QKV projection write its K and V columns straight into
+// cache slot `pos` of each of the m sequences (4-bit: quantized, bit-exact
+// with launch_kv_append on the same fp16 rows; 16-bit: the fp16 values)
+// instead of storing them;
+// LnFuse makes the layer LayerNorm its finished rows [m][n] into `y` after a
+// grid-wide barrier (the launch is cooperative; `sync` = two ints of device
+// memory that are zero on entry and left zero).
+struct KvFuse {
+  uint8_t* k_codes;   // KvView layout of the m sequences' rows (bits == 16:
+  uint32_t* v_words;  // fp16 K / V rows, metas unused)
+  __half2* k_meta;
+  __half2* v_meta;
+  int h, heads, d, max_len, pos, bits;
+};
+struct LnFuse {
+  const __half* g;
+  const __half* b;
+  __half* y;
+  int ldy;
+  float eps;
+  int* sync;
 };
 struct LinearArgs {
   const __half* x; int ldx;       // activations [m][k]
@@ -84,19 +111,52 @@ struct LinearArgs {
   int epi;
   int force_splits;               // 0 = automatic
   int force_tok_tile;             // 0 = automatic
+  const KvFuse* kv;               // decode QKV: quantize K/V into the cache
+  const LnFuse* ln;               // decode out-proj / FC2: LayerNorm of the output rows
+  // Split-tile counters that are zero on entry (and left zero by the
+  // kernel), linear_counter_bytes of them; ws then holds only the partial
+  // tiles.  NULL: the counters follow the partials in ws and are zeroed on
+  // the stream by the launch.
+  int* counters;
 };
+// Largest m the fused decode variants take (one token tile).
+constexpr int kFuseMaxRows = 256;
 size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits);
 cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
 
 // attention
+// Decode attention.  With part/ctr (a 4-bit cache only): when b * heads
+// CTAs cannot fill the GPU, each (sequence, head) is split over several CTAs
+// along the cache, partial results go to `part`
+// (attn_decode_partial_bytes) and the last split of each merges them;
+// ctr = b * heads ints, zero on entry and left zero.
 cudaError_t launch_attn_decode(const __half* q, int ldq, const KvView& kv, int b, int heads, int d,
-                               int kv_bits, int len, __half* out, int ldo, cudaStream_t s);
+                               int kv_bits, int len, __half* out, int ldo, float* part, int* ctr,
+                               cudaStream_t s);
+int attn_decode_splits(int b, int heads, int len);
+// Top-k sparse decode attention over a 4-bit cache: kk keys kept per
+// (sequence, head); idx (optional) receives the kept slots [b][heads][kk] in
+// ascending order.
+cudaError_t launch_attn_topk(const __half* q, int ldq, const KvView& kv, int b, int heads, int d, int len, int kk,
+                             __half* out, int ldo, int32_t* idx, cudaStream_t s);
+// ceil(len * permille / 1000), clamped to 1..len.
+inline int topk_count(int len, int permille) {
+  const long long k = (static_cast<long long>(len) * permille + 999) / 1000;
+  return static_cast<int>(k < 1 ? 1 : (k > len ? len : k));
+}
+size_t attn_decode_partial_bytes(int b, int heads, int d);
 cudaError_t launch_attn_prefill(const __half* qkv, int ldqkv, int b, int seq, int heads, int d,
                                 __half* out, int ldo, cudaStream_t s);
 
 // embedding and greedy choice
-cudaError_t launch_embed(const int32_t* tok, int ld_tok, int b, int ntok, const __half* E, int vocab,
-                         const __half* P, int pos0, int h, __half* x, cudaStream_t s);
+// E: fp16 [vocab][h] (embed_bits 16) or the 4-bit tiled layout (embed_bits 4).
+cudaError_t launch_embed(const int32_t* tok, int ld_tok, int b, int ntok, const void* E, int embed_bits,
+                         int vocab, const __half* P, int pos0, int h, __half* x, cudaStream_t s);
+// Decode embedding of one token per sequence fused with the first layer's
+// LN1: x = E[tok] + P[pos] (fp16) and u = LN(x) (gamma g, beta bta).
+cudaError_t launch_embed_ln(const int32_t* tok, int ld_tok, int b, const void* E, int embed_bits, int vocab,
+                            const __half* P, int pos, int h, __half* x, const __half* g,
+                            const __half* bta, float eps, __half* u, cudaStream_t s);
 cudaError_t launch_argmax(const float* logits, int rows, int vocab, int ld, int32_t* out,
                           int ld_out, cudaStream_t s);
 

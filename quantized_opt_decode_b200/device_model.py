@@ -20,7 +20,8 @@ LINEAR = ("w_qkv", "w_o", "w_fc1", "w_fc2")
 
 def make_config(p: dict) -> fq.flexq_config:
     return fq.flexq_config(h=p["h"], heads=p["heads"], ffn=p["ffn"], w_bits=p["w_bits"],
-                           kv_bits=p["kv_bits"], ln_eps=1e-5)
+                           kv_bits=p["kv_bits"], ln_eps=1e-5,
+                           attn_topk_permille=p.get("topk_permille", 0))
 
 
 def fill_normal(t: torch.Tensor, seed: int, tid: int, sigma: float = 0.02, mean: float = 0.0,
@@ -106,11 +107,18 @@ class DeviceModel:
                        for i in range(self.nl)]
         del scratch
         self.max_pos = max_len
+        self.embed_bits = preset.get("embed_bits", 16)
         self.E = torch.empty(preset["vocab"], cfg.h, dtype=torch.float16, device=device)
         self.P = torch.empty(max_len, cfg.h, dtype=torch.float16, device=device)
         self.lnf_g = torch.empty(cfg.h, dtype=torch.float16, device=device)
         self.lnf_b = torch.empty(cfg.h, dtype=torch.float16, device=device)
         fill_normal(self.E, self.seed, synth.TID_EMBED, stream=stream)
+        if self.embed_bits == 4:
+            # the tied embedding in the linear layers' 4-bit tiled layout
+            packed = torch.empty(fq.flexq_packed_weight_bytes(preset["vocab"], cfg.h), dtype=torch.uint8,
+                                 device=device)
+            fq.flexq_quantize_weight_q4(self.E, preset["vocab"], cfg.h, packed, stream)
+            self.E = packed
         fill_normal(self.P, self.seed, synth.TID_POS, stream=stream)
         fill_normal(self.lnf_g, self.seed, synth.TID_LNF_G, 0.02, 1.0, stream)
         fill_normal(self.lnf_b, self.seed, synth.TID_LNF_B, stream=stream)
@@ -121,7 +129,7 @@ class DeviceModel:
             if self.kv else None
         self.struct = fq.flexq_model(cfg, self.nl, preset["vocab"], max_len, self._layer_arr,
                                      self._kv_arr, self.E.data_ptr(), self.P.data_ptr(),
-                                     self.lnf_g.data_ptr(), self.lnf_b.data_ptr())
+                                     self.lnf_g.data_ptr(), self.lnf_b.data_ptr(), self.embed_bits)
 
     def weight_bytes(self) -> int:
         return sum(t.numel() * t.element_size() for L in self.layers for t in L.t.values())

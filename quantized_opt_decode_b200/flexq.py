@@ -41,7 +41,7 @@ VP = C.c_void_p
 
 class flexq_config(C.Structure):
     _fields_ = [("h", C.c_int), ("heads", C.c_int), ("ffn", C.c_int), ("w_bits", C.c_int),
-                ("kv_bits", C.c_int), ("ln_eps", C.c_float)]
+                ("kv_bits", C.c_int), ("ln_eps", C.c_float), ("attn_topk_permille", C.c_int)]
 
 
 class flexq_layer(C.Structure):
@@ -58,7 +58,7 @@ class flexq_model(C.Structure):
     _fields_ = [("cfg", flexq_config), ("layers", C.c_int), ("vocab", C.c_int),
                 ("max_pos", C.c_int), ("layer", C.POINTER(flexq_layer)),
                 ("kv", C.POINTER(flexq_kv)), ("embed", VP), ("pos_embed", VP), ("lnf_g", VP),
-                ("lnf_b", VP)]
+                ("lnf_b", VP), ("embed_bits", C.c_int)]
 
 
 class flexq_timing(C.Structure):
@@ -92,6 +92,8 @@ _SIGS = {
                          VP], C.c_int),
     "flexq_attention_decode": ([_CFG, C.POINTER(flexq_kv), VP, C.c_int, C.c_int, C.c_int, VP,
                                 C.c_int, VP], C.c_int),
+    "flexq_attention_decode_topk": ([_CFG, C.POINTER(flexq_kv), VP, C.c_int, C.c_int, C.c_int, C.c_int,
+                                     VP, C.c_int, VP, VP], C.c_int),
     "flexq_attention_prefill": ([_CFG, VP, C.c_int, C.c_int, C.c_int, VP, C.c_int, VP], C.c_int),
     "flexq_layer_workspace": ([_CFG, C.c_int, C.c_int], C.c_size_t),
     "flexq_layer_prefill": ([_CFG, C.POINTER(flexq_layer), VP, VP, C.POINTER(flexq_kv), C.c_int,
@@ -219,6 +221,11 @@ def flexq_kv_append(cfg, kv, k, v, ld, b, pos0, ntok, stream=None):
 def flexq_attention_decode(cfg, kv, q, ldq, b, length, out, ldo, stream=None):
     _check(_lib.flexq_attention_decode(C.byref(cfg), C.byref(kv), _p(q), ldq, b, length, _p(out),
                                        ldo, _s(stream)))
+
+
+def flexq_attention_decode_topk(cfg, kv, q, ldq, b, length, k, out, ldo, idx=None, stream=None):
+    _check(_lib.flexq_attention_decode_topk(C.byref(cfg), C.byref(kv), _p(q), ldq, b, length, k,
+                                            _p(out), ldo, _p(idx), _s(stream)))
 
 
 def flexq_attention_prefill(cfg, qkv, ldqkv, b, s, out, ldo, stream=None):

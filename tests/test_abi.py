@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(fq):
 
 
 def test_version_and_empty_error(fq):
-    assert fq.flexq_version() == 100
+    assert fq.flexq_version() == 101
 
 
 def _status(fn, *args):
@@ -69,7 +69,9 @@ def test_packed_weight_size(fq):
 
 def test_config_validation(fq):
     bad = [dict(h=100, heads=1), dict(h=256, heads=3), dict(h=256, heads=1),
-           dict(h=256, heads=4, ffn=100), dict(h=256, heads=4, w_bits=8)]
+           dict(h=256, heads=4, ffn=100), dict(h=256, heads=4, w_bits=8),
+           dict(attn_topk_permille=1001), dict(attn_topk_permille=-1),
+           dict(kv_bits=16, attn_topk_permille=100)]
     for over in bad:
         kw = dict(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=4, ln_eps=1e-5)
         kw.update(over)
@@ -118,10 +120,15 @@ def test_generate_rejects_indivisible_gpu_batch(fq):
     ptrs = [0x10000 * (i + 1) for i in range(12)]
     layer = (fq.flexq_layer * 1)(fq.flexq_layer(*ptrs))
     kv = (fq.flexq_kv * 1)(fq.flexq_kv(0x100000, 0x200000, None, None, 4, 40))
-    m = fq.flexq_model(cfg, 1, 512, 40, layer, kv, 0x1000, 0x2000, 0x3000, 0x4000)
+    m = fq.flexq_model(cfg, 1, 512, 40, layer, kv, 0x1000, 0x2000, 0x3000, 0x4000, 16)
     st = fq._lib.flexq_generate(C.byref(m), 0x5000, 4, 32, 8, 3, 0x6000, 0x7000, 1 << 30, None,
                                 None)
     assert st == 1 and "gpu_batch" in fq.flexq_last_error()
+    m.embed_bits = 8
+    st = fq._lib.flexq_generate(C.byref(m), 0x5000, 4, 32, 8, 4, 0x6000, 0x7000, 1 << 30, None,
+                                None)
+    assert st == 1 and "embed_bits" in fq.flexq_last_error()
+    m.embed_bits = 16
     # s + n - 1 = 41 positions exceed max_pos = 40
     st = fq._lib.flexq_generate(C.byref(m), 0x5000, 4, 32, 10, 4, 0x6000, 0x7000, 1 << 30, None,
                                 None)

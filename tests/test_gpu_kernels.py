@@ -178,3 +178,55 @@ def test_attention_prefill(h, heads, b, s):
     Q, K, V = (opt.heads_split(x[..., i * h:(i + 1) * h], heads) for i in range(3))
     ref = opt.heads_merge(opt.attention_causal(Q, K, V)).reshape(b * s, h)
     assert_close(to_host(out), ref, TOL, what=f"prefill attention s={s}")
+
+
+@pytest.mark.parametrize("h,heads,length,permille", [(512, 4, 545, 100), (256, 4, 37, 100), (1024, 8, 1030, 100),
+                                                     (512, 4, 200, 1000), (256, 4, 64, 10), (512, 4, 1, 100)])
+def test_attention_decode_topk(h, heads, length, permille):
+    """Top-k sparse attention against the oracle on the same 4-bit cache.
+    The kept set is decided from scores, so it is unique only where the k-th
+    and (k+1)-th largest scores are apart by more than the scores' rounding:
+    for those heads the kept slots must equal the oracle's exactly and the
+    output must meet the parity bar; for a head with a near-tie at the
+    threshold the kept set must still be a valid top-k (k slots, each scoring
+    at least the oracle's k-th score minus the margin)."""
+    cfg = _cfg(h, heads, 4)
+    b, L = 3, length + 3
+    d = h // heads
+    rng = np.random.default_rng(length + h + permille)
+    hist = rng.standard_normal((b * length, 3 * h)).astype(np.float16)
+    dev = _dev_cache(cfg, b, L)
+    hd = to_dev(hist)
+    fq.flexq_kv_append(cfg, dev.struct, hd[:, h:], hd[:, 2 * h:], 3 * h, b, 0, length)
+    q = rng.standard_normal((b, 3 * h)).astype(np.float16)
+    kk = opt.topk_count(length, permille)
+    out = torch.empty(b, h, dtype=torch.float16, device="cuda")
+    idx = torch.full((b, heads, kk), -1, dtype=torch.int32, device="cuda")
+    fq.flexq_attention_decode_topk(cfg, dev.struct, to_dev(q), 3 * h, b, length, kk, out, h, idx)
+    fq.flexq_device_status()
+    ocfg = opt.Config(layers=1, h=h, heads=heads, ffn=4 * h, vocab=8, w_bits=4, kv_bits=4)
+    oc = opt.KVCache(ocfg, b, L, 4)
+    oc.write("k", hist[:, h:2 * h].reshape(b, length, h), 0)
+    oc.write("v", hist[:, 2 * h:].reshape(b, length, h), 0)
+    qq = q[:, :h].astype(np.float64).reshape(b, heads, d)
+    K, V = oc.read("k", length), oc.read("v", length)
+    ref, sel = opt.attention_topk(qq, K, V, kk)
+    sc = np.einsum("bad,bald->bal", qq, K) / math.sqrt(d)
+    got_idx = to_host(idx)
+    got = to_host(out).reshape(b, heads, d)
+    clear_got, clear_ref, n_clear = [], [], 0
+    for i in range(b):
+        for j in range(heads):
+            s = np.sort(sc[i, j])[::-1]
+            margin = 1e-3 * np.abs(s).max() + 1e-6
+            gi = got_idx[i, j]
+            assert np.all(np.diff(gi) > 0) and gi.min() >= 0 and gi.max() < length
+            if kk == length or s[kk - 1] - s[kk] > margin:
+                assert np.array_equal(gi, sel[i, j]), (i, j)
+                clear_got.append(got[i, j])
+                clear_ref.append(ref[i, j])
+                n_clear += 1
+            else:
+                assert np.all(sc[i, j][gi] >= s[kk - 1] - margin), (i, j)
+    assert n_clear >= 0.9 * b * heads
+    assert_close(np.stack(clear_got), np.stack(clear_ref), TOL, what=f"top-k attention L={length}")

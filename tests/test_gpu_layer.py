@@ -94,9 +94,11 @@ def test_layer_prefill_and_decode(name, over):
         assert rel_fro(kc[:, :, :s + 1], cache.t["k"][:, :, :s + 1].astype(np.float64)) < TOL
 
 
-@pytest.mark.parametrize("name", ["tiny", "tiny16"])
-def test_generate_tokens_valid_under_oracle(name):
-    p = _preset(name)
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny16", {}),
+                                       ("tiny", dict(embed_bits=4)),        # 4-bit tied embedding / LM head
+                                       ("tiny", dict(topk_permille=100))])  # top-10 % sparse decode attention
+def test_generate_tokens_valid_under_oracle(name, over):
+    p = _preset(name, **over)
     b, s, n = p["b"], p["s"], p["n"]
     dm = DeviceModel(p, b=b, max_len=s + n)
     seed = synth.config_seed(p)
@@ -152,3 +154,126 @@ def test_sequence_subset_matches_block():
     out2 = torch.zeros(2, n, dtype=torch.int32, device="cuda")
     fq.flexq_generate(dm.struct, to_dev(pr[1:3]), 2, s, n, 2, out2, ws, ws_n)
     assert np.array_equal(to_host(out2), full[1:3])
+
+
+@pytest.mark.parametrize("name,over,b", [
+    ("tiny", {}, 5),
+    ("tiny", dict(h=512, heads=4, ffn=2048), 3),     # d = 128
+    ("tiny16", {}, 5),
+    ("tiny", dict(h=512, heads=8, ffn=1024), 37),    # three 16-token chunks, the last ragged
+])
+def test_fused_decode_append_bit_exact(name, over, b):
+    """The decode step appends the token's K/V from inside the QKV projection
+    (quantize on append in its epilogue).  The cache slot it writes must be
+    exactly what the oracle's quantizer makes of the fp16 K/V rows of the
+    same projection run unfused (LayerNorm, then the linear layer alone: same
+    kernel, same K split, so the same fp16 rows); fp16 caches hold those rows."""
+    from gpu_helpers import v_words_to_canonical
+    from oracle import q64
+    p = _preset(name, **over)
+    h, a = p["h"], p["heads"]
+    d = h // a
+    pos = 11
+    dm = DeviceModel(p, b=b, max_len=pos + 3, layers=1)
+    rng = np.random.default_rng(b + h)
+    t = rng.standard_normal((b, h)).astype(np.float16)
+    td = to_dev(t)
+    t2 = torch.empty_like(td)
+    ws_n = fq.flexq_layer_workspace(dm.cfg, b, 1)
+    ws = workspace(ws_n)
+    L, kv = dm.layers[0].struct, dm.kv[0].struct
+    fq.flexq_layer_decode(dm.cfg, L, td, t2, kv, b, pos, ws, ws_n)
+    fq.flexq_device_status()
+    # unfused: LN1, then the QKV linear layer alone
+    lw = dm.layers[0].t
+    u = torch.empty_like(td)
+    fq.flexq_layernorm(td, h, lw["ln1_g"], lw["ln1_b"], u, h, b, h, 1e-5)
+    qkv = torch.empty(b, 3 * h, dtype=torch.float16, device="cuda")
+    lin_ws = fq.flexq_linear_workspace(b, 3 * h, h, p["w_bits"], 0)
+    lws = workspace(lin_ws)
+    fq.flexq_linear(u, h, lw["w_qkv"], p["w_bits"], b, 3 * h, h, lw["b_qkv"], None, 0, fq.EPI_BIAS, qkv, 3 * h,
+                    lws, lin_ws, 0)
+    rows = to_host(qkv)
+    K = rows[:, h:2 * h].reshape(b, a, d)
+    V = rows[:, 2 * h:].reshape(b, a, d)
+    L_ = pos + 3
+    if p["kv_bits"] == 4:
+        kc = to_host(dm.kv[0].k).reshape(b, a, L_, d // 2)[:, :, pos]
+        km = to_host(dm.kv[0].k_meta).reshape(b, a, L_, d // 64, 2)[:, :, pos]
+        vm = to_host(dm.kv[0].v_meta).reshape(b, a, L_, d // 64, 2)[:, :, pos]
+        vc = v_words_to_canonical(to_host(dm.kv[0].v), b, a, L_, d)[:, :, pos]
+        for got_c, got_m, rows16 in ((kc, km, K), (vc, vm, V)):
+            c, m, s = q64.quantize_rows(rows16)
+            assert np.array_equal(got_c, c)
+            assert np.array_equal(got_m[..., 0].view(np.uint16), m.view(np.uint16))
+            assert np.array_equal(got_m[..., 1].view(np.uint16), s.view(np.uint16))
+    else:
+        kc = to_host(dm.kv[0].k).reshape(b, a, L_, d)[:, :, pos]
+        vc = to_host(dm.kv[0].v).reshape(b, a, L_, d)[:, :, pos]
+        assert np.array_equal(kc.view(np.uint16), K.view(np.uint16))
+        assert np.array_equal(vc.view(np.uint16), V.view(np.uint16))
+
+
+@pytest.mark.parametrize("name,over,b,length", [
+    ("tiny", dict(h=512, heads=4, ffn=1024), 2, 1100),   # d = 128, cache split over 5 CTAs
+    ("tiny", {}, 3, 1056),                                # d = 64
+    ("tiny", dict(h=512, heads=4, ffn=1024), 1, 300),     # a ragged 128-token chunk per split
+])
+def test_layer_decode_long_cache(name, over, b, length):
+    """Decode over a long 4-bit cache with so few (sequence, head) pairs that
+    the attention splits each head's cache across CTAs and merges the partial
+    softmax results.  The cache is filled from seeded fp16 rows on both sides
+    through the quantizer (bit-exact), then one decode step appends slot
+    `length` and attends over length + 1 slots."""
+    p = _preset(name, **over)
+    h = p["h"]
+    cfg = opt.Config.from_preset(p, ln1_f16=True)
+    seed = synth.config_seed(p)
+    W = opt.effective_layer(cfg, opt.raw_layer(cfg, seed, 0))
+    dm = DeviceModel(p, b=b, max_len=length + 2, layers=1)
+    rng = np.random.default_rng(length + b)
+    rows = rng.standard_normal((b * length, 2 * h)).astype(np.float16)
+    t = rng.standard_normal((b, h)).astype(np.float16)
+    rd = to_dev(rows)
+    kv = dm.kv[0].struct
+    fq.flexq_kv_append(dm.cfg, kv, rd[:, :h], rd[:, h:], 2 * h, b, 0, length)
+    ws_n = fq.flexq_layer_workspace(dm.cfg, b, 1)
+    ws = workspace(ws_n)
+    td = to_dev(t)
+    t2 = torch.empty_like(td)
+    fq.flexq_layer_decode(dm.cfg, dm.layers[0].struct, td, t2, kv, b, length, ws, ws_n)
+    fq.flexq_device_status()
+    cache = opt.KVCache(cfg, b, length + 2, 4)
+    cache.write("k", rows[:, :h].reshape(b, length, h), 0)
+    cache.write("v", rows[:, h:].reshape(b, length, h), 0)
+    ref = opt.layer_decode(cfg, W, t.astype(np.float64), cache, length)
+    _check_out(to_host(t2), ref, t)
+
+
+def test_layer_decode_topk_sparse_attention():
+    """A decode step whose attention keeps the top 10 % of the cache (the
+    configuration's attn_topk_permille), against the oracle's decode with the
+    same option."""
+    p = _preset("tiny", h=512, heads=4, ffn=1024, topk_permille=100)
+    h, b, length = p["h"], 3, 700
+    cfg = opt.Config.from_preset(p, ln1_f16=True)
+    seed = synth.config_seed(p)
+    W = opt.effective_layer(cfg, opt.raw_layer(cfg, seed, 0))
+    dm = DeviceModel(p, b=b, max_len=length + 2, layers=1)
+    rng = np.random.default_rng(71)
+    rows = rng.standard_normal((b * length, 2 * h)).astype(np.float16)
+    t = rng.standard_normal((b, h)).astype(np.float16)
+    rd = to_dev(rows)
+    kv = dm.kv[0].struct
+    fq.flexq_kv_append(dm.cfg, kv, rd[:, :h], rd[:, h:], 2 * h, b, 0, length)
+    ws_n = fq.flexq_layer_workspace(dm.cfg, b, 1)
+    ws = workspace(ws_n)
+    td = to_dev(t)
+    t2 = torch.empty_like(td)
+    fq.flexq_layer_decode(dm.cfg, dm.layers[0].struct, td, t2, kv, b, length, ws, ws_n)
+    fq.flexq_device_status()
+    cache = opt.KVCache(cfg, b, length + 2, 4)
+    cache.write("k", rows[:, :h].reshape(b, length, h), 0)
+    cache.write("v", rows[:, h:].reshape(b, length, h), 0)
+    ref = opt.layer_decode(cfg, W, t.astype(np.float64), cache, length)
+    _check_out(to_host(t2), ref, t)

@@ -515,3 +515,61 @@ def test_ln1_f16_prefill_rounds_projection_input():
                 u = [float(np.float16(v)) for v in u]
             k = _bf_lin(u, W["w_qkv"][cfg.h:2 * cfg.h], W["b_qkv"][cfg.h:2 * cfg.h])
             assert np.array_equal(K[0, r], np.array(k).astype(np.float16))
+
+
+# ---------------------------------------------------------------------------
+# Top-k sparse attention ("FlexGen研究学术报告" section 三(C))
+# ---------------------------------------------------------------------------
+def test_topk_count_is_ten_percent_rounded_up():
+    assert opt.topk_count(528, 100) == 53 and opt.topk_count(10, 100) == 1
+    assert opt.topk_count(1, 100) == 1 and opt.topk_count(7, 1000) == 7 and opt.topk_count(11, 100) == 2
+
+
+def test_topk_selection_brute_force_and_ties():
+    """The kept set is the k largest scores; at a tie the lower index wins:
+    checked against a selection by repeated arg-max in pure Python."""
+    rng = np.random.default_rng(21)
+    for trial in range(50):
+        L = int(rng.integers(1, 40))
+        sc = rng.integers(-4, 5, size=L).astype(float).tolist()  # many ties
+        k = int(rng.integers(1, L + 1))
+        left = list(range(L))
+        want = []
+        for _ in range(k):
+            best = left[0]
+            for t in left:
+                if sc[t] > sc[best]:
+                    best = t  # strict: the first (lowest) index of a tie stays
+            want.append(best)
+            left.remove(best)
+        assert opt.topk_select(sc, k) == sorted(want), (sc, k)
+    assert opt.topk_select([1.0, 3.0, 3.0, 2.0, 3.0], 2) == [1, 2]
+
+
+def test_topk_attention_brute_force_and_limits(rng):
+    b, a, L, d = 2, 2, 23, 16
+    q = rng.standard_normal((b, a, d))
+    k = rng.standard_normal((b, a, L, d))
+    v = rng.standard_normal((b, a, L, d))
+    kk = opt.topk_count(L, 100)
+    got, sel = opt.attention_topk(q, k, v, kk)
+    for i in range(b):
+        for j in range(a):
+            sc = [sum(q[i, j, e] * k[i, j, t, e] for e in range(d)) / math.sqrt(d) for t in range(L)]
+            m = max(sc)
+            z = sum(math.exp(x - m) for x in sc)
+            keep = sorted(range(L), key=lambda t: (-sc[t], t))[:kk]
+            assert sorted(keep) == sel[i, j].tolist()
+            ref = [sum(math.exp(sc[t] - m) / z * v[i, j, t, e] for t in keep) for e in range(d)]
+            assert np.allclose(got[i, j], ref, rtol=1e-12, atol=1e-12)
+    # k = L is dense attention; k = 1 keeps the arg-max key with its full-softmax weight
+    dense, _ = opt.attention_topk(q, k, v, L)
+    assert np.allclose(dense, opt.attention_single(q, k, v), rtol=1e-13, atol=1e-13)
+    one, sel1 = opt.attention_topk(q, k, v, 1)
+    sc = np.einsum("bad,bald->bal", q, k) / math.sqrt(d)
+    p = opt.softmax(sc)
+    top = sc.argmax(axis=-1)
+    assert np.array_equal(sel1[..., 0], top)
+    for i in range(b):
+        for j in range(a):
+            assert np.allclose(one[i, j], p[i, j, top[i, j]] * v[i, j, top[i, j]], rtol=1e-13)
