@@ -621,6 +621,105 @@ def run_flexq(args, p):
         dist.destroy_process_group()
 
 
+def measure_h2d_gbps(torch, stream, nbytes=1 << 30, reps=5):
+    """Page-locked host to device copy rate (GB/s), CUDA events on `stream`."""
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    with torch.cuda.stream(stream):
+        dst.copy_(src, non_blocking=True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            dst.copy_(src, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    return nbytes * reps / (e0.elapsed_time(e1) / 1e3) / 1e9
+
+
+def run_offload(args, p):
+    """Decode throughput with the layer weights in page-locked host memory:
+    the block (GPU batch x GPU batches) chosen by the library's cost model
+    from the measured host-to-device rate and the measured device peaks; one
+    step = one flexq_generate_offload (prefill column + n-1 decode columns),
+    decode tokens/s from its device-timed decode phase."""
+    import torch
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    from quantized_opt_decode_b200 import build
+    build.build()
+    from quantized_opt_decode_b200 import flexq as fq
+    from quantized_opt_decode_b200.device_model import DeviceModel, workspace
+
+    s, n = p["s"], p["n"]
+    stream, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d = measure_h2d_gbps(torch, copy)
+    t_setup = time.perf_counter()
+    with torch.cuda.stream(stream):
+        dm = DeviceModel(p, b=0, max_len=s + n, stream=stream, with_kv=False, offload=True)
+    stream.synchronize()
+    torch.cuda.empty_cache()
+    peaks = load_peaks()
+    free, _ = torch.cuda.mem_get_info()
+    hw = fq.flexq_hw(h2d_gbps=h2d, hbm_gbps=peaks["hbm_gbps"], tensor_tflops=peaks["bf16_tflops_sustained"],
+                     device_bytes=free - 6e9)
+    ch = fq.flexq_offload_plan(dm.struct, s, n, hw, args.max_block)
+    gbs, b = ch.gpu_batch, ch.gpu_batch * ch.num_batches
+    dm.alloc_kv(b, s + n)
+    prompts = torch.empty(b, s, dtype=torch.int32, device="cuda")
+    fq.flexq_synth_tokens(prompts, b * s, synth.config_seed(p), synth.TID_PROMPT, p["vocab"], stream=stream)
+    out = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+    ws_n = fq.flexq_generate_workspace(dm.struct, b, s, gbs)
+    ws = workspace(ws_n)
+    slot = fq.flexq_offload_slot_bytes(dm.cfg)
+    slots = workspace(2 * slot)
+    stream.synchronize()
+    setup_s = time.perf_counter() - t_setup
+
+    def step():
+        t = fq.flexq_timing()
+        fq.flexq_generate_offload(dm.struct, slots, 2 * slot, copy, prompts, b, s, n, gbs, out, ws, ws_n, t, stream)
+        return t.prefill_ms, t.decode_ms
+
+    for _ in range(args.warmup):
+        step()
+    fq.flexq_device_status(stream)
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clk:
+        torch.cuda.synchronize()
+        l0 = fq.flexq_launch_count()
+        times = [step() for _ in range(args.steps)]
+        launches = fq.flexq_launch_count() - l0
+    fq.flexq_device_status(stream)
+    pre = sum(t[0] for t in times) / len(times)
+    dec = sum(t[1] for t in times) / len(times)
+    w_bytes = sum(dm.layers[0].t[k].numel() * dm.layers[0].t[k].element_size() for k in
+                  ("w_qkv", "w_o", "w_fc1", "w_fc2")) * p["layers"]
+    line = {
+        "metric": METRIC, "mode": "offloaded weights", "value": round(b * (n - 1) / (dec / 1e3), 2),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dec, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic (seeded splitmix64 draws; weights ~N(0,0.02) quantized to 4-bit)",
+        "config": {"workload": workload_name(args) + "+offload", "layers": p["layers"], "h": p["h"],
+                   "global_batch": b, "gpu_batch": gbs, "seq_len": s, "gen_tokens": n,
+                   "w_bits": p["w_bits"], "kv_bits": p["kv_bits"],
+                   "weights": f"page-locked host memory, {w_bytes / 1e9:.1f} GB, two device slots",
+                   "step": "one flexq_generate_offload; value from its decode phase (n-1 columns)"},
+        "plan": {"gpu_batch": gbs, "num_batches": ch.num_batches, "max_block": args.max_block,
+                 "modelled_decode_tokens_per_s": round(ch.decode_tokens_per_s, 1),
+                 "modelled_column_io_s": round(ch.column_io_s, 4),
+                 "modelled_column_compute_s": round(ch.column_compute_s, 4),
+                 "modelled_device_gb": round(ch.device_bytes / 1e9, 1),
+                 "h2d_gbps_measured": round(h2d, 1)},
+        "measured_column_ms": round(dec / (n - 1), 2),
+        "link_frac": round(w_bytes / (dec / (n - 1) / 1e3) / (h2d * 1e9), 4),
+        "generation_tokens_per_s": round(b * n / ((pre + dec) / 1e3), 2),
+        "prefill_ms": round(pre, 1),
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+        "setup_s": round(setup_s, 1),
+        "kernel_sources": csrc_hash(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -632,6 +731,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-codec", action="store_true")
+    ap.add_argument("--offload", action="store_true",
+                    help="layer weights in page-locked host memory, block chosen by the cost model")
+    ap.add_argument("--max-block", type=int, default=288, help="largest block the offload plan may choose")
     ap.add_argument("--embed-bits", type=int, default=16, choices=[16, 4],
                     help="4: tied embedding / LM head stored group-wise 4-bit")
     ap.add_argument("--topk", type=int, default=0,
@@ -646,6 +748,8 @@ def main():
         p["topk_permille"] = args.topk
     if args.impl == "reference":
         run_reference(args, p)
+    elif args.offload:
+        run_offload(args, p)
     else:
         run_flexq(args, p)
 

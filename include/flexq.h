@@ -351,6 +351,62 @@ flexq_status flexq_generate(const flexq_model* model, const int32_t* prompt_dev,
                             flexq_timing* timing, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Offloaded weights ([WT] "Search Space", "Cost Model"; [RPT] 三(A)/(B)).     */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of one device slot holding a layer's four weight matrices
+ * (qkv, o, fc1, fc2 in that order, each 256-byte aligned). */
+size_t flexq_offload_slot_bytes(const flexq_config* cfg);
+
+/* flexq_generate with the layer weights resident in host memory: every
+ * model->layer[i].w_qkv / w_o / w_fc1 / w_fc2 points into page-locked host
+ * memory (checked; FLEXQ_ERR_INVALID otherwise), every other pointer of the
+ * model is device memory.  Each column of the zig-zag block (the prefill,
+ * then each decode step) walks the layers in order and runs every GPU batch
+ * of the block on one layer before the next, so each layer's weights cross
+ * the host link once per column: they are copied into one of two device
+ * slots (slots_dev: 2 * flexq_offload_slot_bytes bytes, caller-owned) on
+ * copy_stream (a stream other than `stream`) two layer steps ahead of the
+ * compute on `stream`, overlapping the copy of the next layer with this
+ * layer's compute.  Results equal flexq_generate's on the same weights.
+ * The call returns once all work is enqueued (with timing, once it ends). */
+flexq_status flexq_generate_offload(const flexq_model* model, void* slots_dev, size_t slots_bytes,
+                                    void* copy_stream, const int32_t* prompt_dev, int b, int s, int n,
+                                    int gpu_batch, int32_t* out_dev, void* ws_dev, size_t ws_bytes,
+                                    flexq_timing* timing, void* stream);
+
+typedef struct {
+  double h2d_gbps;      /* host-to-device copy rate (GB/s), measured by the caller */
+  double hbm_gbps;      /* device memory rate (GB/s) */
+  double tensor_tflops; /* dense fp16 tensor rate (TFLOP/s) */
+  double device_bytes;  /* device memory the generation may use */
+} flexq_hw;
+
+typedef struct {
+  int gpu_batch;               /* sequences per GPU batch */
+  int num_batches;             /* GPU batches per block: b = gpu_batch * num_batches */
+  double decode_tokens_per_s;  /* modelled decode throughput of the choice */
+  double column_io_s;          /* modelled weight-copy time of one decode column */
+  double column_compute_s;     /* modelled compute time of one decode column */
+  double device_bytes;         /* modelled device memory of the choice */
+} flexq_offload_choice;
+
+/* Cost model of the offloaded block schedule: per decode column and layer,
+ * T = max(weight bytes / h2d, num_batches * t_batch) with t_batch the
+ * roofline time of one GPU batch's layer step at the mean KV length s + n/2
+ * (weights and KV at hbm_gbps, 2 * tokens * weights flops at tensor_tflops),
+ * plus the LM head once per column; throughput = b / column time.  Device
+ * memory = two weight slots, E, P, biases and LayerNorms, every layer's KV
+ * cache for b sequences of s + n slots and flexq_generate_workspace.
+ * Enumerates gpu_batch = 256, 240, .., 16 and num_batches = 1, 2, .. while
+ * the memory fits and b <= max_block, and returns the highest modelled
+ * throughput; a later candidate replaces the best only when it is more than
+ * 0.1 % faster, so among near-equal choices the larger GPU batch (the more
+ * efficient GEMMs) and then the smaller block win. */
+flexq_status flexq_offload_plan(const flexq_model* model, int s, int n, const flexq_hw* hw, int max_block,
+                                flexq_offload_choice* out);
+
+/* ------------------------------------------------------------------------ */
 /* Instrumentation (measurement only; not part of the method).                */
 /* ------------------------------------------------------------------------ */
 

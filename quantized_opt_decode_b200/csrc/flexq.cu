@@ -794,10 +794,114 @@ flexq_status lm_head(const flexq_model* m, const __half* x_last, int ldx, int b,
   return FLEXQ_OK;
 }
 
+// Where a column's layer weights come from.  Resident: the model's own
+// device pointers.  Offloaded ([WT] "Search Space": the zig-zag block
+// schedule loads a layer's weights once per column and reuses them for every
+// GPU batch of the block; [RPT] 三(A)): the four weight matrices of every
+// layer stay in page-locked host memory and are copied into one of two
+// device slots on a copy stream two (column, layer) steps ahead of the
+// compute stream, so the copy of the next layer overlaps this layer's
+// compute; events order each slot's reuse.
+struct LayerFeed {
+  const flexq_model* m = nullptr;
+  bool offload = false;
+  uint8_t* slots = nullptr;
+  size_t slot_bytes = 0;
+  size_t off[4] = {};
+  size_t bytes[4] = {};
+  cudaStream_t copy = nullptr, compute = nullptr;
+  cudaEvent_t copied[2] = {}, freed[2] = {};
+  flexq_layer slot_layer[2] = {};
+  long long step = 0, total = 0;  // (column, layer) steps taken / to take in this call
+
+  explicit LayerFeed(const flexq_model* model) : m(model) {}
+  LayerFeed(const LayerFeed&) = delete;
+  ~LayerFeed() {
+    for (int i = 0; i < 2; ++i) {
+      if (copied[i]) cudaEventDestroy(copied[i]);
+      if (freed[i]) cudaEventDestroy(freed[i]);
+    }
+  }
+
+  flexq_status copy_step(long long g) {
+    const int slot = static_cast<int>(g & 1);
+    const flexq_layer& L = m->layer[g % m->layers];
+    const void* src[4] = {L.w_qkv, L.w_o, L.w_fc1, L.w_fc2};
+    FQ_CUDA(cudaStreamWaitEvent(copy, freed[slot], 0), "wait for a free weight slot");
+    for (int i = 0; i < 4; ++i)
+      FQ_CUDA(cudaMemcpyAsync(slots + slot * slot_bytes + off[i], src[i], bytes[i], cudaMemcpyHostToDevice, copy),
+              "weight copy to the device");
+    FQ_CUDA(cudaEventRecord(copied[slot], copy), "event record");
+    return FLEXQ_OK;
+  }
+
+  flexq_status start(long long steps) {
+    total = steps;
+    step = 0;
+    if (!offload) return FLEXQ_OK;
+    for (int i = 0; i < 2; ++i) {
+      FQ_CUDA(cudaEventCreateWithFlags(&copied[i], cudaEventDisableTiming), "event create");
+      FQ_CUDA(cudaEventCreateWithFlags(&freed[i], cudaEventDisableTiming), "event create");
+      // nothing has used the slot yet: its first copy need not wait
+      FQ_CUDA(cudaEventRecord(freed[i], compute), "event record");
+    }
+    for (long long g = 0; g < std::min<long long>(2, total); ++g) FQ_TRY(copy_step(g));
+    return FLEXQ_OK;
+  }
+
+  // The layer to run at this step (waits for its weights when offloaded).
+  const flexq_layer* begin(int l, flexq_status* st) {
+    *st = FLEXQ_OK;
+    if (!offload) return &m->layer[l];
+    const int slot = static_cast<int>(step & 1);
+    const cudaError_t e = cudaStreamWaitEvent(compute, copied[slot], 0);
+    if (e != cudaSuccess) {
+      *st = cuda_fail(e, "wait for layer weights");
+      return nullptr;
+    }
+    slot_layer[slot] = m->layer[l];
+    uint8_t* base = slots + slot * slot_bytes;
+    slot_layer[slot].w_qkv = base + off[0];
+    slot_layer[slot].w_o = base + off[1];
+    slot_layer[slot].w_fc1 = base + off[2];
+    slot_layer[slot].w_fc2 = base + off[3];
+    return &slot_layer[slot];
+  }
+
+  flexq_status end() {
+    if (offload) {
+      const int slot = static_cast<int>(step & 1);
+      FQ_CUDA(cudaEventRecord(freed[slot], compute), "event record");
+      if (step + 2 < total) FQ_TRY(copy_step(step + 2));
+    }
+    ++step;
+    return FLEXQ_OK;
+  }
+};
+
+// Bytes of one matrix as the layer stores it.
+size_t weight_bytes(const flexq_config* c, int n_out, int k_in) {
+  return c->w_bits == 4 ? flexq_packed_weight_bytes(n_out, k_in) : static_cast<size_t>(n_out) * k_in * 2;
+}
+
+// Offsets of a layer's four weight matrices in a device slot; returns the
+// slot's size.
+size_t slot_layout(const flexq_config* c, size_t off[4], size_t bytes[4]) {
+  const size_t b[4] = {weight_bytes(c, 3 * c->h, c->h), weight_bytes(c, c->h, c->h), weight_bytes(c, c->ffn, c->h),
+                       weight_bytes(c, c->h, c->ffn)};
+  size_t o = 0;
+  for (int i = 0; i < 4; ++i) {
+    off[i] = o;
+    bytes[i] = b[i];
+    o += align_up(b[i]);
+  }
+  return o;
+}
+
 // Prefill column of the zig-zag block: every layer over every GPU batch,
 // then the first token of each sequence.
 flexq_status prefill_column(const flexq_model* model, const int32_t* prompt_dev, int b, int s, int n, int gpu_batch,
-                            int32_t* out_dev, const GenWs& w, cudaStream_t st) {
+                            int32_t* out_dev, const GenWs& w, cudaStream_t st, LayerFeed& feed) {
   const flexq_config* c = &model->cfg;
   const int h = c->h, nb = b / gpu_batch;
   {
@@ -809,11 +913,14 @@ flexq_status prefill_column(const flexq_model* model, const int32_t* prompt_dev,
   __half *x = w.x, *y = w.y;
   const LayerWs lw = layer_ws_layout(c, gpu_batch * s, w.layer);
   for (int l = 0; l < model->layers; ++l) {
+    flexq_status fs;
+    const flexq_layer* L = feed.begin(l, &fs);
+    FQ_TRY(fs);
     for (int k = 0; k < nb; ++k) {
       const size_t off = static_cast<size_t>(k) * gpu_batch * s * h;
-      FQ_TRY(layer_step(c, &model->layer[l], x + off, y + off, &model->kv[l], k * gpu_batch, gpu_batch, s, 0, true,
-                        lw, st));
+      FQ_TRY(layer_step(c, L, x + off, y + off, &model->kv[l], k * gpu_batch, gpu_batch, s, 0, true, lw, st));
     }
+    FQ_TRY(feed.end());
     std::swap(x, y);
   }
   return lm_head(model, x + static_cast<size_t>(s - 1) * h, s * h, b, w, out_dev, n, st);
@@ -822,7 +929,7 @@ flexq_status prefill_column(const flexq_model* model, const int32_t* prompt_dev,
 // Decode columns j = 1 .. n-1: the token in out[:, j-1] at position s+j-1
 // runs through every layer for every GPU batch and yields out[:, j].
 flexq_status decode_columns(const flexq_model* model, int b, int s, int n, int gpu_batch, int32_t* out_dev,
-                            const GenWs& w, cudaStream_t st) {
+                            const GenWs& w, cudaStream_t st, LayerFeed& feed) {
   const flexq_config* c = &model->cfg;
   const int h = c->h, nb = b / gpu_batch;
   const LayerWs lw = layer_ws_layout(c, gpu_batch, w.layer);
@@ -847,11 +954,15 @@ flexq_status decode_columns(const flexq_model* model, int b, int s, int n, int g
         const bool last = l + 1 == model->layers;
         const void* g = last ? model->lnf_g : model->layer[l + 1].ln1_g;
         const void* bb = last ? model->lnf_b : model->layer[l + 1].ln1_b;
+        flexq_status fs;
+        const flexq_layer* L = feed.begin(l, &fs);
+        FQ_TRY(fs);
         for (int k = 0; k < nb; ++k) {
           const size_t off = static_cast<size_t>(k) * gpu_batch * h;
-          FQ_TRY(decode_fused(c, &model->layer[l], t + off, w.tn + off, t2 + off, w.tn + off, g, bb, &model->kv[l],
-                              k * gpu_batch, gpu_batch, pos, lw, st));
+          FQ_TRY(decode_fused(c, L, t + off, w.tn + off, t2 + off, w.tn + off, g, bb, &model->kv[l], k * gpu_batch,
+                              gpu_batch, pos, lw, st));
         }
+        FQ_TRY(feed.end());
         std::swap(t, t2);
       }
       FQ_TRY(lm_head(model, w.tn, h, b, w, out_dev + j, n, st, true));
@@ -868,11 +979,14 @@ flexq_status decode_columns(const flexq_model* model, int b, int s, int n, int g
     }
     __half *t = w.t, *t2 = w.t2;
     for (int l = 0; l < model->layers; ++l) {
+      flexq_status fs;
+      const flexq_layer* L = feed.begin(l, &fs);
+      FQ_TRY(fs);
       for (int k = 0; k < nb; ++k) {
         const size_t off = static_cast<size_t>(k) * gpu_batch * h;
-        FQ_TRY(layer_step(c, &model->layer[l], t + off, t2 + off, &model->kv[l], k * gpu_batch, gpu_batch, 1, pos,
-                          false, lw, st));
+        FQ_TRY(layer_step(c, L, t + off, t2 + off, &model->kv[l], k * gpu_batch, gpu_batch, 1, pos, false, lw, st));
       }
+      FQ_TRY(feed.end());
       std::swap(t, t2);
     }
     FQ_TRY(lm_head(model, t, h, b, w, out_dev + j, n, st));
@@ -891,30 +1005,34 @@ flexq_status flexq_generate_prefill(const flexq_model* model, const int32_t* pro
   GenWs w;
   FQ_TRY(check_generation(model, b, s, n, gpu_batch, out_dev, ws_dev, ws_bytes, &w));
   FQ_CHECK(prompt_dev != nullptr, "NULL prompt pointer");
-  return prefill_column(model, prompt_dev, b, s, n, gpu_batch, out_dev, w, as_stream(stream));
+  LayerFeed feed(model);
+  FQ_TRY(feed.start(model->layers));
+  return prefill_column(model, prompt_dev, b, s, n, gpu_batch, out_dev, w, as_stream(stream), feed);
 }
 
 flexq_status flexq_generate_decode(const flexq_model* model, int b, int s, int n, int gpu_batch, int32_t* out_dev,
                                    void* ws_dev, size_t ws_bytes, void* stream) {
   GenWs w;
   FQ_TRY(check_generation(model, b, s, n, gpu_batch, out_dev, ws_dev, ws_bytes, &w));
-  return decode_columns(model, b, s, n, gpu_batch, out_dev, w, as_stream(stream));
+  LayerFeed feed(model);
+  FQ_TRY(feed.start(static_cast<long long>(n - 1) * model->layers));
+  return decode_columns(model, b, s, n, gpu_batch, out_dev, w, as_stream(stream), feed);
 }
 
-flexq_status flexq_generate(const flexq_model* model, const int32_t* prompt_dev, int b, int s, int n, int gpu_batch,
-                            int32_t* out_dev, void* ws_dev, size_t ws_bytes, flexq_timing* timing, void* stream) {
-  GenWs w;
-  FQ_TRY(check_generation(model, b, s, n, gpu_batch, out_dev, ws_dev, ws_bytes, &w));
-  FQ_CHECK(prompt_dev != nullptr, "NULL prompt pointer");
-  cudaStream_t st = as_stream(stream);
+namespace {
+// The whole generation (prefill column, n-1 decode columns) with the given
+// layer feed; fills timing when asked.
+flexq_status generate_all(const flexq_model* model, const int32_t* prompt_dev, int b, int s, int n, int gpu_batch,
+                          int32_t* out_dev, const GenWs& w, flexq_timing* timing, cudaStream_t st, LayerFeed& feed) {
   cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
   if (timing) {
     for (auto& e : ev) FQ_CUDA(cudaEventCreate(&e), "event create");
     FQ_CUDA(cudaEventRecord(ev[0], st), "event record");
   }
-  flexq_status rc = prefill_column(model, prompt_dev, b, s, n, gpu_batch, out_dev, w, st);
+  flexq_status rc = feed.start(static_cast<long long>(n) * model->layers);
+  if (rc == FLEXQ_OK) rc = prefill_column(model, prompt_dev, b, s, n, gpu_batch, out_dev, w, st, feed);
   if (rc == FLEXQ_OK && timing) cudaEventRecord(ev[1], st);
-  if (rc == FLEXQ_OK) rc = decode_columns(model, b, s, n, gpu_batch, out_dev, w, st);
+  if (rc == FLEXQ_OK) rc = decode_columns(model, b, s, n, gpu_batch, out_dev, w, st, feed);
   if (timing) {
     if (rc == FLEXQ_OK) {
       cudaEventRecord(ev[2], st);
@@ -926,6 +1044,102 @@ flexq_status flexq_generate(const flexq_model* model, const int32_t* prompt_dev,
       if (e) cudaEventDestroy(e);
   }
   return rc;
+}
+}  // namespace
+
+flexq_status flexq_generate(const flexq_model* model, const int32_t* prompt_dev, int b, int s, int n, int gpu_batch,
+                            int32_t* out_dev, void* ws_dev, size_t ws_bytes, flexq_timing* timing, void* stream) {
+  GenWs w;
+  FQ_TRY(check_generation(model, b, s, n, gpu_batch, out_dev, ws_dev, ws_bytes, &w));
+  FQ_CHECK(prompt_dev != nullptr, "NULL prompt pointer");
+  LayerFeed feed(model);
+  return generate_all(model, prompt_dev, b, s, n, gpu_batch, out_dev, w, timing, as_stream(stream), feed);
+}
+
+// --- offloaded weights --------------------------------------------------------------
+size_t flexq_offload_slot_bytes(const flexq_config* cfg) {
+  if (check_config(cfg) != FLEXQ_OK) return 0;
+  size_t off[4], bytes[4];
+  return slot_layout(cfg, off, bytes);
+}
+
+flexq_status flexq_generate_offload(const flexq_model* model, void* slots_dev, size_t slots_bytes, void* copy_stream,
+                                    const int32_t* prompt_dev, int b, int s, int n, int gpu_batch, int32_t* out_dev,
+                                    void* ws_dev, size_t ws_bytes, flexq_timing* timing, void* stream) {
+  GenWs w;
+  FQ_TRY(check_generation(model, b, s, n, gpu_batch, out_dev, ws_dev, ws_bytes, &w));
+  FQ_CHECK(prompt_dev != nullptr, "NULL prompt pointer");
+  FQ_CHECK(copy_stream != stream, "the weight copies need a stream of their own");
+  LayerFeed feed(model);
+  feed.offload = true;
+  feed.slot_bytes = slot_layout(&model->cfg, feed.off, feed.bytes);
+  FQ_CHECK(slots_dev != nullptr && aligned16(slots_dev), "slots must be a 16-byte aligned device buffer");
+  if (slots_bytes < 2 * feed.slot_bytes)
+    return fail(FLEXQ_ERR_WORKSPACE, "offload needs %zu slot bytes, got %zu", 2 * feed.slot_bytes, slots_bytes);
+  for (int i = 0; i < model->layers; ++i) {
+    const flexq_layer& L = model->layer[i];
+    for (const void* p : {L.w_qkv, L.w_o, L.w_fc1, L.w_fc2}) {
+      cudaPointerAttributes attr{};
+      const cudaError_t e = cudaPointerGetAttributes(&attr, p);
+      if (e != cudaSuccess) cudaGetLastError();
+      FQ_CHECK(e == cudaSuccess && attr.type == cudaMemoryTypeHost,
+               "layer %d: offloaded weights must be page-locked host memory", i);
+    }
+  }
+  feed.slots = static_cast<uint8_t*>(slots_dev);
+  feed.copy = as_stream(copy_stream);
+  feed.compute = as_stream(stream);
+  return generate_all(model, prompt_dev, b, s, n, gpu_batch, out_dev, w, timing, feed.compute, feed);
+}
+
+flexq_status flexq_offload_plan(const flexq_model* model, int s, int n, const flexq_hw* hw, int max_block,
+                                flexq_offload_choice* out) {
+  FQ_CHECK(model != nullptr && hw != nullptr && out != nullptr, "NULL pointer");
+  FQ_TRY(check_config(&model->cfg));
+  FQ_CHECK(model->layers > 0 && model->vocab > 0, "model needs layers and a vocabulary");
+  FQ_CHECK(s > 0 && n > 0 && max_block > 0, "s, n and max_block must be positive");
+  FQ_CHECK(hw->h2d_gbps > 0 && hw->hbm_gbps > 0 && hw->tensor_tflops > 0 && hw->device_bytes > 0,
+           "hardware rates and memory must be positive");
+  const flexq_config* c = &model->cfg;
+  const double h = c->h, ffn = c->ffn, L = model->layers;
+  size_t off[4], bytes[4];
+  const double slot = static_cast<double>(slot_layout(c, off, bytes));
+  const double w_layer = static_cast<double>(bytes[0] + bytes[1] + bytes[2] + bytes[3]);
+  const double flop_tok = 2.0 * (4.0 * h * h + 2.0 * h * ffn);  // 2 * (QKV + out + FC1 + FC2) per token
+  const double kv_row = static_cast<double>(flexq_kv_bytes(c, 1, 1024)) / 1024.0 / 2.0;  // K or V bytes per slot
+  const double lbar = s + n / 2.0;
+  const double bw = hw->hbm_gbps * 1e9, tc = hw->tensor_tflops * 1e12, io_bw = hw->h2d_gbps * 1e9;
+  const double e_bytes = model->embed_bits == 4 ? static_cast<double>(flexq_packed_weight_bytes(model->vocab, c->h))
+                                                : static_cast<double>(model->vocab) * h * 2;
+  const double fixed = 2.0 * slot + e_bytes + static_cast<double>(model->max_pos) * h * 2 + L * (16.0 * h + 2 * ffn);
+  flexq_offload_choice best{};
+  best.decode_tokens_per_s = -1.0;
+  // larger GPU batches first: among choices within 0.1 % of each other the
+  // model cannot tell apart, the larger batch runs the more efficient GEMMs
+  for (int gbs = kFuseMaxRows; gbs >= 16; gbs -= 16) {
+    for (int nb = 1; static_cast<long long>(gbs) * nb <= max_block; ++nb) {
+      const int b = gbs * nb;
+      const double mem = fixed + L * static_cast<double>(flexq_kv_bytes(c, b, s + n)) +
+                         static_cast<double>(flexq_generate_workspace(model, b, s, gbs));
+      if (mem > hw->device_bytes) break;  // a larger block only needs more
+      const double batch = std::max(w_layer / bw, flop_tok * gbs / tc) + gbs * lbar * 2.0 * kv_row / bw;
+      const double io = w_layer / io_bw, comp = nb * batch;
+      const double head = std::max(e_bytes / bw, 2.0 * b * model->vocab * h / tc);
+      const double column = L * std::max(io, comp) + head;
+      const double tps = b / column;
+      if (tps > best.decode_tokens_per_s * 1.001) {
+        best.gpu_batch = gbs;
+        best.num_batches = nb;
+        best.decode_tokens_per_s = tps;
+        best.column_io_s = L * io;
+        best.column_compute_s = L * comp + head;
+        best.device_bytes = mem;
+      }
+    }
+  }
+  FQ_CHECK(best.gpu_batch > 0, "no block of at least 16 sequences fits in %.3g device bytes", hw->device_bytes);
+  *out = best;
+  return FLEXQ_OK;
 }
 
 // --- instrumentation -------------------------------------------------------------

@@ -61,10 +61,11 @@ class KVCache:
 
 
 class DeviceLayer:
-    """One decoder layer's parameters on the device."""
+    """One decoder layer's parameters on the device (with offload=True the four
+    weight matrices end up in page-locked host memory instead)."""
 
     def __init__(self, cfg: fq.flexq_config, seed: int, layer: int, scratch: torch.Tensor | None,
-                 device="cuda", stream=None):
+                 device="cuda", stream=None, offload: bool = False):
         self.t = {}
         for name in synth.LAYER_TENSORS:
             shape, sigma, mean = synth.layer_tensor_spec(name, cfg.h, cfg.ffn)
@@ -83,6 +84,14 @@ class DeviceLayer:
                 buf = torch.empty(shape, dtype=torch.float16, device=device)
                 fill_normal(buf, seed, tid, sigma, mean, stream)
                 self.t[name] = buf
+            if offload and name in LINEAR:
+                dev = self.t[name]
+                host = torch.empty(dev.shape, dtype=dev.dtype, pin_memory=True)
+                if stream is not None:
+                    stream.synchronize()
+                host.copy_(dev)
+                self.t[name] = host
+                del dev
         self.struct = fq.flexq_layer(*[self.t[n].data_ptr() for n in (
             "w_qkv", "w_o", "w_fc1", "w_fc2", "b_qkv", "b_o", "b_fc1", "b_fc2",
             "ln1_g", "ln1_b", "ln2_g", "ln2_b")])
@@ -93,7 +102,7 @@ class DeviceModel:
     a block of b sequences of up to max_len positions."""
 
     def __init__(self, preset: dict, b: int, max_len: int, layers: int | None = None,
-                 device="cuda", stream=None, with_kv: bool = True):
+                 device="cuda", stream=None, with_kv: bool = True, offload: bool = False):
         self.p = preset
         self.cfg = make_config(preset)
         self.seed = synth.config_seed(preset)
@@ -103,7 +112,8 @@ class DeviceModel:
         if cfg.w_bits == 4:
             scratch = torch.empty(max(3 * cfg.h * cfg.h, cfg.ffn * cfg.h), dtype=torch.float16,
                                   device=device)
-        self.layers = [DeviceLayer(cfg, self.seed, i, scratch, device, stream)
+        self.offload = offload
+        self.layers = [DeviceLayer(cfg, self.seed, i, scratch, device, stream, offload)
                        for i in range(self.nl)]
         del scratch
         self.max_pos = max_len
@@ -122,12 +132,18 @@ class DeviceModel:
         fill_normal(self.P, self.seed, synth.TID_POS, stream=stream)
         fill_normal(self.lnf_g, self.seed, synth.TID_LNF_G, 0.02, 1.0, stream)
         fill_normal(self.lnf_b, self.seed, synth.TID_LNF_B, stream=stream)
-        self.kv = [KVCache(cfg, b, max_len, device) for _ in range(self.nl)] if with_kv else []
-        self.b = b
+        self.device = device
         self._layer_arr = (fq.flexq_layer * self.nl)(*[L.struct for L in self.layers])
+        self.alloc_kv(b if with_kv else 0, max_len)
+
+    def alloc_kv(self, b: int, max_len: int):
+        """(Re)allocates every layer's KV cache for b sequences (none for 0)."""
+        self.kv = []
+        self.kv = [KVCache(self.cfg, b, max_len, self.device) for _ in range(self.nl)] if b > 0 else []
+        self.b = b
         self._kv_arr = (fq.flexq_kv * max(1, len(self.kv)))(*[k.struct for k in self.kv]) \
             if self.kv else None
-        self.struct = fq.flexq_model(cfg, self.nl, preset["vocab"], max_len, self._layer_arr,
+        self.struct = fq.flexq_model(self.cfg, self.nl, self.p["vocab"], self.max_pos, self._layer_arr,
                                      self._kv_arr, self.E.data_ptr(), self.P.data_ptr(),
                                      self.lnf_g.data_ptr(), self.lnf_b.data_ptr(), self.embed_bits)
 

@@ -65,6 +65,16 @@ class flexq_timing(C.Structure):
     _fields_ = [("prefill_ms", C.c_float), ("decode_ms", C.c_float)]
 
 
+class flexq_hw(C.Structure):
+    _fields_ = [("h2d_gbps", C.c_double), ("hbm_gbps", C.c_double), ("tensor_tflops", C.c_double),
+                ("device_bytes", C.c_double)]
+
+
+class flexq_offload_choice(C.Structure):
+    _fields_ = [("gpu_batch", C.c_int), ("num_batches", C.c_int), ("decode_tokens_per_s", C.c_double),
+                ("column_io_s", C.c_double), ("column_compute_s", C.c_double), ("device_bytes", C.c_double)]
+
+
 _CFG = C.POINTER(flexq_config)
 _SIGS = {
     "flexq_last_error": ([], C.c_char_p),
@@ -108,6 +118,11 @@ _SIGS = {
                                 VP, C.c_size_t, VP], C.c_int),
     "flexq_generate_decode": ([C.POINTER(flexq_model), C.c_int, C.c_int, C.c_int, C.c_int, VP, VP,
                                C.c_size_t, VP], C.c_int),
+    "flexq_offload_slot_bytes": ([_CFG], C.c_size_t),
+    "flexq_generate_offload": ([C.POINTER(flexq_model), VP, C.c_size_t, VP, VP, C.c_int, C.c_int, C.c_int,
+                                C.c_int, VP, VP, C.c_size_t, C.POINTER(flexq_timing), VP], C.c_int),
+    "flexq_offload_plan": ([C.POINTER(flexq_model), C.c_int, C.c_int, C.POINTER(flexq_hw), C.c_int,
+                            C.POINTER(flexq_offload_choice)], C.c_int),
     "flexq_launch_count": ([], C.c_uint64),
     "flexq_profile_start": ([], C.c_int),
     "flexq_profile_stop": ([VP, C.POINTER(C.c_float), C.POINTER(C.c_int)], C.c_int),
@@ -266,6 +281,23 @@ def flexq_generate_prefill(model, prompt, b, s, n, gpu_batch, out, ws, ws_bytes,
 def flexq_generate_decode(model, b, s, n, gpu_batch, out, ws, ws_bytes, stream=None):
     _check(_lib.flexq_generate_decode(C.byref(model), b, s, n, gpu_batch, _p(out), _p(ws),
                                       ws_bytes, _s(stream)))
+
+
+def flexq_offload_slot_bytes(cfg) -> int:
+    return _lib.flexq_offload_slot_bytes(C.byref(cfg))
+
+
+def flexq_generate_offload(model, slots, slots_bytes, copy_stream, prompt, b, s, n, gpu_batch, out, ws,
+                           ws_bytes, timing=None, stream=None):
+    _check(_lib.flexq_generate_offload(C.byref(model), _p(slots), slots_bytes, _s(copy_stream), _p(prompt), b,
+                                       s, n, gpu_batch, _p(out), _p(ws), ws_bytes,
+                                       C.byref(timing) if timing is not None else None, _s(stream)))
+
+
+def flexq_offload_plan(model, s, n, hw, max_block):
+    choice = flexq_offload_choice()
+    _check(_lib.flexq_offload_plan(C.byref(model), s, n, C.byref(hw), max_block, C.byref(choice)))
+    return choice
 
 
 def flexq_launch_count() -> int:

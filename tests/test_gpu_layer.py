@@ -277,3 +277,35 @@ def test_layer_decode_topk_sparse_attention():
     cache.write("v", rows[:, h:].reshape(b, length, h), 0)
     ref = opt.layer_decode(cfg, W, t.astype(np.float64), cache, length)
     _check_out(to_host(t2), ref, t)
+
+
+@pytest.mark.parametrize("gbs", [4, 2])
+def test_offloaded_weights_match_resident(gbs):
+    """Generation with the layer weights in page-locked host memory, copied
+    into two device slots on a second stream ahead of the compute, gives the
+    tokens of the resident run bit for bit (same kernels, same weights; only
+    where the weights come from differs)."""
+    p = _preset("tiny", b=4)
+    b, s, n = 4, p["s"], 6
+    seed = synth.config_seed(p)
+    prompts = to_dev(synth.tokens(seed, synth.TID_PROMPT, b * s, p["vocab"]).reshape(b, s))
+    res = DeviceModel(p, b=b, max_len=s + n)
+    off = DeviceModel(p, b=b, max_len=s + n, offload=True)
+    assert off.layers[0].t["w_qkv"].device.type == "cpu" and off.layers[0].t["w_qkv"].is_pinned()
+    ws_n = fq.flexq_generate_workspace(res.struct, b, s, gbs)
+    ws = workspace(ws_n)
+    out_r = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+    fq.flexq_generate(res.struct, prompts, b, s, n, gbs, out_r, ws, ws_n)
+    slot = fq.flexq_offload_slot_bytes(off.cfg)
+    slots = workspace(2 * slot)
+    copy = torch.cuda.Stream()
+    out_o = torch.zeros(b, n, dtype=torch.int32, device="cuda")
+    timing = fq.flexq_timing()
+    fq.flexq_generate_offload(off.struct, slots, 2 * slot, copy, prompts, b, s, n, gbs, out_o, ws, ws_n, timing)
+    fq.flexq_device_status()
+    assert np.array_equal(to_host(out_o), to_host(out_r))
+    assert timing.prefill_ms > 0 and timing.decode_ms > 0
+    # weights that are not page-locked host memory are refused
+    with pytest.raises(fq.FlexqError) as ei:
+        fq.flexq_generate_offload(res.struct, slots, 2 * slot, copy, prompts, b, s, n, gbs, out_o, ws, ws_n)
+    assert ei.value.status == 1 and "page-locked" in str(ei.value)
