@@ -5,7 +5,9 @@
 
 Kernels: qkv, out_proj, fc1, fc2 (dequant-fused linear layers at the decode
 batch, or --rows for prefill-sized inputs), attn_decode (one layer's 4-bit
-cache at KV length s + n/2), attn_prefill, kv_append, layernorm, lm_head.
+cache at KV length s + n/2), attn_topk (the same cache, top-k sparse),
+layer_decode (one fused decode layer step), attn_prefill, kv_append,
+layernorm, lm_head.
 Prints one JSON line per kernel: average device time over --reps launches
 (CUDA events on the launching stream, after --warmup launches) and the
 achieved rate of the method's algorithmic bytes or FLOPs.  Also the small
@@ -91,10 +93,9 @@ def bench_gemm(p, kind, M, reps, warmup, stream, splits):
     return ms, byts, flops, {"M": M, "N": n, "K": k}
 
 
-def bench_attn_decode(p, b, reps, warmup, stream):
-    cfg = make_config(p)
-    h, a = p["h"], p["heads"]
-    L = p["s"] + p["n"] // 2
+def _filled_cache(p, cfg, b, L, stream):
+    """One layer's cache for b sequences holding L seeded rows each."""
+    h = p["h"]
     kv = KVCache(cfg, b, L + 1)
     seed = synth.config_seed(p)
     chunk = max(1, (1 << 28) // (b * 3 * h * 2))  # rows of history per fill pass
@@ -104,18 +105,61 @@ def bench_attn_decode(p, b, reps, warmup, stream):
         fq.flexq_synth_normal_f16(rows, b * nt * 3 * h, seed, 997, t0 * 3 * h, 1.0, 0.0, stream)
         fq.flexq_kv_append(cfg, kv.struct, rows[:, h:], rows[:, 2 * h:], 3 * h, b, t0, nt, stream)
     del rows
+    return kv
+
+
+def bench_attn_decode(p, b, reps, warmup, stream, topk=0):
+    cfg = make_config(p)
+    h, a = p["h"], p["heads"]
+    L = p["s"] + p["n"] // 2
+    kv = _filled_cache(p, cfg, b, L, stream)
+    seed = synth.config_seed(p)
     q = torch.empty(b, 3 * h, dtype=torch.float16, device="cuda")
     fq.flexq_synth_normal_f16(q, b * 3 * h, seed, 996, 0, 1.0, 0.0, stream)
     out = torch.empty(b, h, dtype=torch.float16, device="cuda")
 
+    kk = max(1, -(-L * topk // 1000))
+
     def run():
-        fq.flexq_attention_decode(cfg, kv.struct, q, 3 * h, b, L, out, h, stream)
+        if topk:
+            fq.flexq_attention_decode_topk(cfg, kv.struct, q, 3 * h, b, L, kk, out, h, None, stream)
+        else:
+            fq.flexq_attention_decode(cfg, kv.struct, q, 3 * h, b, L, out, h, stream)
 
     ms = _time(run, reps, warmup, stream)
     d = h // a
     row = (d / 2 + 4 * d / 64) if p["kv_bits"] == 4 else 2 * d
-    byts = b * a * L * 2 * row + 2 * b * h * 2
-    return ms, byts, 4.0 * b * L * h, {"b": b, "L": L, "heads": a, "d": d}
+    # top-k: every key, the kept keys' values (the method's bytes)
+    byts = b * a * (L + (kk if topk else L)) * row + 2 * b * h * 2
+    return ms, byts, 2.0 * b * (L + (kk if topk else L)) * h, {"b": b, "L": L, "heads": a, "d": d, "kept": kk}
+
+
+def bench_layer_decode(p, b, reps, warmup, stream):
+    """One fused decode layer step (QKV with the KV append, attention,
+    output projection with LN2, FC1, FC2) at KV length s + n/2."""
+    from .device_model import DeviceLayer
+    cfg = make_config(p)
+    h = p["h"]
+    L = p["s"] + p["n"] // 2
+    seed = synth.config_seed(p)
+    layer = DeviceLayer(cfg, seed, 0, None, "cuda", stream)
+    kv = _filled_cache(p, cfg, b, L, stream)
+    t = torch.empty(b, h, dtype=torch.float16, device="cuda")
+    fq.flexq_synth_normal_f16(t, b * h, seed, 991, 0, 1.0, 0.0, stream)
+    y = torch.empty_like(t)
+    ws_n = fq.flexq_layer_workspace(cfg, b, 1)
+    ws = workspace(ws_n)
+
+    def run():
+        fq.flexq_layer_decode(cfg, layer.struct, t, y, kv.struct, b, L, ws, ws_n, stream)
+
+    ms = _time(run, reps, warmup, stream)
+    wb = 0.5 + 4 / 64 if p["w_bits"] == 4 else 2.0
+    d = h // p["heads"]
+    row = (d / 2 + 4 * d / 64) if p["kv_bits"] == 4 else 2 * d
+    byts = (4 * h * h + 2 * h * p["ffn"]) * wb + b * p["heads"] * (L + 1) * 2 * row
+    flops = 2.0 * b * (4 * h * h + 2 * h * p["ffn"]) + 4.0 * b * (L + 1) * h
+    return ms, byts, flops, {"b": b, "L": L + 1}
 
 
 def bench_attn_prefill(p, b, reps, warmup, stream):
@@ -188,6 +232,7 @@ def main():
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--topk", type=int, default=100, help="attn_topk: keys kept per mille")
     a = ap.parse_args()
     p = dict(synth.CONFIGS[a.config])
     hbm, tf = _peaks()
@@ -201,6 +246,10 @@ def main():
                                                     stream, a.splits)
             elif kind == "attn_decode":
                 ms, byts, flops, shape = bench_attn_decode(p, p["gpu_batch"], a.reps, a.warmup, stream)
+            elif kind == "attn_topk":
+                ms, byts, flops, shape = bench_attn_decode(p, p["gpu_batch"], a.reps, a.warmup, stream, a.topk)
+            elif kind == "layer_decode":
+                ms, byts, flops, shape = bench_layer_decode(p, p["gpu_batch"], a.reps, a.warmup, stream)
             elif kind == "attn_prefill":
                 ms, byts, flops, shape = bench_attn_prefill(p, max(1, p["gpu_batch"] // 8), a.reps, a.warmup,
                                                             stream)
