@@ -279,8 +279,8 @@ flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* lay
  * K/V columns straight into the cache: the same codes flexq_kv_append gives
  * those fp16 rows), LN2 runs inside the output projection (a cooperative
  * launch whose CTAs normalise the finished rows after a grid-wide barrier),
- * and decode attention over a 4-bit cache splits each head's cache over
- * several CTAs when b * heads CTAs would not fill the GPU. */
+ * and decode attention splits each head's cache over several CTAs when
+ * b * heads CTAs would not fill the GPU. */
 flexq_status flexq_layer_decode(const flexq_config* cfg, const flexq_layer* layer,
                                 const void* t_dev, void* y_dev, const flexq_kv* kv, int b,
                                 int pos, void* ws_dev, size_t ws_bytes, void* stream);

@@ -5,12 +5,9 @@
 // survey notes' eq. (2), with K and V stored in the group-wise 4-bit format of
 // "FlexGen研究学术报告" section 三(C) (or fp16).
 //
-// Two kernels.  The fp16 cache: one CTA per (head, sequence), 4 warps, 8
-// tokens per warp in flight with 4 lanes per token; pass 1 writes the scores
-// to shared memory and finds their maximum, pass 2 exponentiates, pass 3
-// streams V.  The 4-bit cache (below): a pipelined kernel that streams each
-// head's rows through shared memory.  In both, 4-bit codes are dequantized
-// without materialising x_hat:
+// Two pipelined kernels, one per cache format, that stream each head's rows
+// through shared memory (below).  4-bit codes are dequantized without
+// materialising x_hat:
 //   q . x_hat = scale * sum_e q_e code_e + min * sum_e q_e   (per group)
 //   sum_t p_t x_hat_t = sum_t (p_t scale_t) code_t + sum_t p_t min_t,
 // which is the dequantized value code * scale + min before its fp16 rounding.
@@ -24,164 +21,6 @@
 
 namespace flexq {
 namespace {
-
-constexpr int kThreads = 128;
-
-__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
-  v = is_max ? warp_max(v) : warp_sum(v);
-  const int w = threadIdx.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[w] = v;
-  __syncthreads();
-  float r = red[0];
-#pragma unroll
-  for (int i = 1; i < kThreads / 32; ++i) r = is_max ? fmaxf(r, red[i]) : r + red[i];
-  return r;
-}
-
-// Loads this lane's d/4 elements of one cached row as fp32 "codes" (4-bit) or
-// values (16-bit).
-template <int D, int KV_BITS>
-__device__ __forceinline__ void load_row_part(const void* base, size_t slot, int c, float (&x)[D / 4]) {
-  constexpr int DPL = D / 4;
-  if constexpr (KV_BITS == 4) {
-    const uint8_t* p = static_cast<const uint8_t*>(base) + slot * (D / 2) + c * (DPL / 2);
-    uint32_t w[DPL / 8];
-    if constexpr (DPL == 32) {
-      const uint4 u = *reinterpret_cast<const uint4*>(p);
-      w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
-    } else {
-      const uint2 u = *reinterpret_cast<const uint2*>(p);
-      w[0] = u.x; w[1] = u.y;
-    }
-#pragma unroll
-    for (int j = 0; j < DPL / 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[j * 8 + e] = static_cast<float>((w[j] >> (4 * e)) & 0xF);
-  } else {
-    const __half* p = static_cast<const __half*>(base) + slot * D + c * DPL;
-#pragma unroll
-    for (int j = 0; j < DPL / 8; ++j) {
-      const uint4 u = reinterpret_cast<const uint4*>(p)[j];
-      const __half2* h2 = reinterpret_cast<const __half2*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h2[e]);
-        x[j * 8 + 2 * e] = f.x;
-        x[j * 8 + 2 * e + 1] = f.y;
-      }
-    }
-  }
-}
-
-template <int D, int KV_BITS>
-__global__ void __launch_bounds__(kThreads) attn_decode_kernel(const __half* __restrict__ q, int ldq,
-                                                               KvView kv, int heads, int len,
-                                                               __half* __restrict__ out, int ldo,
-                                                               float inv_sqrt_d) {
-  constexpr int DPL = D / 4;
-  extern __shared__ float sc[];
-  __shared__ float red[kThreads / 32];
-  __shared__ float part[kThreads / 32][D + 4];
-  const int j = blockIdx.x, i = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = lane & 3;
-  const int g = (c * DPL) / 64;  // group of this lane's dimensions
-  const size_t row0 = (static_cast<size_t>(i) * heads + j) * kv.max_len;
-
-  float qf[DPL];
-  const __half* qp = q + static_cast<size_t>(i) * ldq + j * D + c * DPL;
-#pragma unroll
-  for (int e = 0; e < DPL; e += 2) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(qp + e));
-    qf[e] = f.x;
-    qf[e + 1] = f.y;
-  }
-  float qsum = 0.f;
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) qsum += qf[e];
-
-  // pass 1: scores
-  float mx = -INFINITY;
-  for (int base = warp * 8; base < len; base += kThreads / 4) {
-    const int t = base + (lane >> 2);
-    const bool valid = t < len;
-    float partial = 0.f;
-    if (valid) {
-      float x[DPL];
-      load_row_part<D, KV_BITS>(kv.k, row0 + t, c, x);
-      float dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) dot = fmaf(qf[e], x[e], dot);
-      if constexpr (KV_BITS == 4) {
-        const __half2 ms = static_cast<const __half2*>(kv.k_meta)[(row0 + t) * (D / 64) + g];
-        const float2 f = __half22float2(ms);  // (min, scale)
-        partial = f.y * dot + f.x * qsum;
-      } else {
-        partial = dot;
-      }
-    }
-    partial += __shfl_xor_sync(0xffffffffu, partial, 1);
-    partial += __shfl_xor_sync(0xffffffffu, partial, 2);
-    if (valid) {
-      const float s = partial * inv_sqrt_d;
-      if (c == 0) sc[t] = s;
-      mx = fmaxf(mx, s);
-    }
-  }
-  const float M = block_reduce(mx, red, true);
-
-  // pass 2: exponentials (scores were written before the reduction's barrier)
-  float sum = 0.f;
-  for (int t = threadIdx.x; t < len; t += kThreads) {
-    const float p = __expf(sc[t] - M);
-    sc[t] = p;
-    sum += p;
-  }
-  const float S = block_reduce(sum, red, false);
-
-  // pass 3: weighted sum of V
-  float acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  float am = 0.f;
-  for (int base = warp * 8; base < len; base += kThreads / 4) {
-    const int t = base + (lane >> 2);
-    if (t < len) {
-      const float p = sc[t];
-      float x[DPL];
-      load_row_part<D, KV_BITS>(kv.v, row0 + t, c, x);
-      float w = p;
-      if constexpr (KV_BITS == 4) {
-        const float2 f = __half22float2(static_cast<const __half2*>(kv.v_meta)[(row0 + t) * (D / 64) + g]);
-        w = p * f.y;
-        am = fmaf(p, f.x, am);
-      }
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, x[e], acc[e]);
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) {
-    float v = acc[e] + am;
-    v += __shfl_xor_sync(0xffffffffu, v, 4);
-    v += __shfl_xor_sync(0xffffffffu, v, 8);
-    v += __shfl_xor_sync(0xffffffffu, v, 16);
-    acc[e] = v;
-  }
-  if (lane < 4) {
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) part[warp][c * DPL + e] = acc[e];
-  }
-  __syncthreads();
-  const float invS = 1.0f / S;
-  for (int e = threadIdx.x; e < D; e += kThreads) {
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) v += part[w][e];
-    out[static_cast<size_t>(i) * ldo + j * D + e] = __float2half_rn(v * invS);
-  }
-}
 
 // ---------------------------------------------------------------------------
 // 4-bit cache: streamed through shared memory, integer dot products.
@@ -264,6 +103,75 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Merges the compute warps' online-softmax states (running max, sum, and
+// weighted value sums) in warp order; with several splits along the cache
+// the merged state goes to `part` and the last split to arrive merges all of
+// them in split order (results independent of timing) and resets the
+// (sequence, head) counter.  Every thread of the CTA calls it after the
+// warps have published cm / cl / cacc.
+template <int D>
+__device__ void merge_and_store(const float* cm, const float* cl, const float (*cacc)[D], __half* __restrict__ out,
+                                int ldo, int i, int j, size_t hr, int z, float* __restrict__ part,
+                                int* __restrict__ ctr, int* last_flag) {
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, cm[w]);
+  float ws[kComputeWarps];
+  float Lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < kComputeWarps; ++w) {
+    ws[w] = cm[w] == -INFINITY ? 0.f : __expf(cm[w] - M);
+    Lsum += cl[w] * ws[w];
+  }
+  const int S = gridDim.z;
+  if (S == 1) {
+    for (int e = threadIdx.x; e < D; e += blockDim.x) {
+      float o = 0.f;
+#pragma unroll
+      for (int w = 0; w < kComputeWarps; ++w) o += cacc[w][e] * ws[w];
+      out[static_cast<size_t>(i) * ldo + j * D + e] = __float2half_rn(o / Lsum);
+    }
+    return;
+  }
+  float* mine = part + (hr * S + z) * (D + 2);
+  for (int e = threadIdx.x; e < D; e += blockDim.x) {
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kComputeWarps; ++w) o += cacc[w][e] * ws[w];
+    __stcg(mine + 2 + e, o);
+  }
+  if (threadIdx.x == 0) {
+    __stcg(mine, M);
+    __stcg(mine + 1, Lsum);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(ctr + hr, 1);
+    *last_flag = old == S - 1;
+    if (*last_flag) ctr[hr] = 0;  // every split has counted in: leave the counter zero
+    __threadfence();
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  const float* all = part + hr * S * (D + 2);
+  float Mz = -INFINITY;
+  for (int zz = 0; zz < S; ++zz) Mz = fmaxf(Mz, __ldcg(all + zz * (D + 2)));
+  float Lz = 0.f;
+  for (int zz = 0; zz < S; ++zz) {
+    const float mz = __ldcg(all + zz * (D + 2));
+    if (mz != -INFINITY) Lz += __ldcg(all + zz * (D + 2) + 1) * __expf(mz - Mz);
+  }
+  for (int e = threadIdx.x; e < D; e += blockDim.x) {
+    float o = 0.f;
+    for (int zz = 0; zz < S; ++zz) {
+      const float mz = __ldcg(all + zz * (D + 2));
+      if (mz != -INFINITY) o += __ldcg(all + zz * (D + 2) + 2 + e) * __expf(mz - Mz);
+    }
+    out[static_cast<size_t>(i) * ldo + j * D + e] = __float2half_rn(o / Lz);
+  }
 }
 
 template <int D>
@@ -519,64 +427,7 @@ __global__ void __launch_bounds__(kQ4Threads) attn_decode_q4_kernel(const __half
   }
   __syncthreads();
 
-  // merge the warps (fixed order), then the splits
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kComputeWarps; ++w) M = fmaxf(M, cm[w]);
-  float ws[kComputeWarps];
-  float Lsum = 0.f;
-#pragma unroll
-  for (int w = 0; w < kComputeWarps; ++w) {
-    ws[w] = cm[w] == -INFINITY ? 0.f : __expf(cm[w] - M);
-    Lsum += cl[w] * ws[w];
-  }
-  const int S = gridDim.z;
-  if (S == 1) {
-    for (int e = threadIdx.x; e < D; e += kQ4Threads) {
-      float o = 0.f;
-#pragma unroll
-      for (int w = 0; w < kComputeWarps; ++w) o += cacc[w][e] * ws[w];
-      out[static_cast<size_t>(i) * ldo + j * D + e] = __float2half_rn(o / Lsum);
-    }
-    return;
-  }
-  float* mine = part + (hr * S + z) * (D + 2);
-  for (int e = threadIdx.x; e < D; e += kQ4Threads) {
-    float o = 0.f;
-#pragma unroll
-    for (int w = 0; w < kComputeWarps; ++w) o += cacc[w][e] * ws[w];
-    __stcg(mine + 2 + e, o);
-  }
-  if (threadIdx.x == 0) {
-    __stcg(mine, M);
-    __stcg(mine + 1, Lsum);
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int old = atomicAdd(ctr + hr, 1);
-    last_flag = old == S - 1;
-    if (last_flag) ctr[hr] = 0;  // every split has counted in: leave the counter zero
-    __threadfence();
-  }
-  __syncthreads();
-  if (!last_flag) return;
-  const float* all = part + hr * S * (D + 2);
-  float Mz = -INFINITY;
-  for (int zz = 0; zz < S; ++zz) Mz = fmaxf(Mz, __ldcg(all + zz * (D + 2)));
-  float Lz = 0.f;
-  for (int zz = 0; zz < S; ++zz) {
-    const float mz = __ldcg(all + zz * (D + 2));
-    if (mz != -INFINITY) Lz += __ldcg(all + zz * (D + 2) + 1) * __expf(mz - Mz);
-  }
-  for (int e = threadIdx.x; e < D; e += kQ4Threads) {
-    float o = 0.f;
-    for (int zz = 0; zz < S; ++zz) {
-      const float mz = __ldcg(all + zz * (D + 2));
-      if (mz != -INFINITY) o += __ldcg(all + zz * (D + 2) + 2 + e) * __expf(mz - Mz);
-    }
-    out[static_cast<size_t>(i) * ldo + j * D + e] = __float2half_rn(o / Lz);
-  }
+  merge_and_store<D>(cm, cl, cacc, out, ldo, i, j, hr, z, part, ctr, &last_flag);
 }
 
 template <int D>
@@ -596,18 +447,189 @@ cudaError_t launch_q4(const __half* q, int ldq, const KvView& kv, int b, int hea
   return launched();
 }
 
-template <int D, int KV_BITS>
-cudaError_t launch_one(const __half* q, int ldq, const KvView& kv, int b, int heads, int len,
-                       __half* out, int ldo, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(len) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel<D, KV_BITS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+// ---------------------------------------------------------------------------
+// fp16 cache: the same pipeline with fp16 K and V rows (T tokens per stage,
+// K rows then V rows, two bulk copies), fp32 dot products and an fp32
+// weighted sum of V per warp.
+// ---------------------------------------------------------------------------
+template <int D>
+struct F16Stage {
+  static constexpr int T = D == 128 ? 64 : 128;  // tokens per chunk
+  static constexpr int row = D * 2;              // bytes per K or V row
+  static constexpr int bytes = 2 * T * row;
+  static constexpr int stages = 3;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kQ4Threads) attn_decode_f16_kernel(const __half* __restrict__ q, int ldq, KvView kv,
+                                                                     int heads, int len, __half* __restrict__ out,
+                                                                     int ldo, float inv_sqrt_d, int span,
+                                                                     float* __restrict__ part, int* __restrict__ ctr,
+                                                                     uint64_t wait_ns, uint32_t* err) {
+  using L = F16Stage<D>;
+  constexpr int T = L::T, NS = L::stages;
+  constexpr int TW = T / kComputeWarps;  // tokens per warp and chunk
+  constexpr int DPL = D / 4;             // score pass: dimensions per lane
+  constexpr int DPV = D / 32;            // value pass: dimensions per lane
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[NS], empty[NS];
+  __shared__ float cm[kComputeWarps], cl[kComputeWarps];
+  __shared__ float cacc[kComputeWarps][D];
+  __shared__ int last_flag;
+  const int j = blockIdx.x, i = blockIdx.y, z = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t hr = static_cast<size_t>(i) * heads + j;
+  const int t_begin = z * span;
+  const int t_end = min(len, t_begin + span);
+  const int n_chunks = t_end > t_begin ? (t_end - t_begin + T - 1) / T : 0;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < NS; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], kComputeWarps);
+    }
+    mbar_fence_init();
   }
-  dim3 grid(heads, b);
-  attn_decode_kernel<D, KV_BITS><<<grid, kThreads, smem, s>>>(q, ldq, kv, heads, len, out, ldo,
-                                                              1.0f / sqrtf(static_cast<float>(D)));
+  __syncthreads();
+
+  if (warp == kComputeWarps) {
+    if (lane == 0) {
+      // every (sequence, head) row block is contiguous and 16-byte aligned
+      const uint8_t* kb = static_cast<const uint8_t*>(kv.k) + hr * kv.max_len * L::row;
+      const uint8_t* vb = static_cast<const uint8_t*>(kv.v) + hr * kv.max_len * L::row;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int st = c % NS;
+        if (!mbar_wait(&empty[st], (static_cast<uint32_t>(c / NS) & 1u) ^ 1u, wait_ns)) {
+          set_error(err, DEV_TIMEOUT_PRODUCER);
+          break;
+        }
+        const int t0 = t_begin + c * T;
+        const uint32_t bytes = static_cast<uint32_t>(min(T, t_end - t0)) * L::row;
+        uint8_t* sb = ring + st * L::bytes;
+        mbar_arrive_expect_tx(&full[st], 2 * bytes);
+        bulk_g2s(sb, kb + static_cast<size_t>(t0) * L::row, bytes, &full[st]);
+        bulk_g2s(sb + T * L::row, vb + static_cast<size_t>(t0) * L::row, bytes, &full[st]);
+      }
+      const uint64_t drain = wait_ns > 1000000000ull ? wait_ns : 1000000000ull;
+      for (int c = max(0, n_chunks - NS); c < n_chunks; ++c)
+        mbar_wait(&full[c % NS], static_cast<uint32_t>(c / NS) & 1u, drain);
+    }
+  } else {
+    const int tk = lane >> 2, cq = lane & 3;
+    float qf[DPL];
+    const __half* qp = q + static_cast<size_t>(i) * ldq + j * D + cq * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(qp + e));
+      qf[e] = f.x;
+      qf[e + 1] = f.y;
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    float acc[DPV];
+#pragma unroll
+    for (int e = 0; e < DPV; ++e) acc[e] = 0.f;
+    bool bad = false;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int st = c % NS;
+      if (!bad && !mbar_wait(&full[st], static_cast<uint32_t>(c / NS) & 1u, wait_ns)) {
+        set_error(err, DEV_TIMEOUT_CONSUMER);
+        bad = true;
+      }
+      const int nt = min(T, t_end - (t_begin + c * T));
+      const __half* sk = reinterpret_cast<const __half*>(ring + st * L::bytes);
+      const __half* sv = sk + T * D;
+      const int wt0 = warp * TW;
+      float sc[TW / 8];
+      float mloc = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < TW / 8; ++u) {
+        const int tt = wt0 + u * 8 + tk;
+        const bool valid = !bad && tt < nt;
+        float partial = 0.f;
+        if (valid) {
+          const uint4* kr = reinterpret_cast<const uint4*>(sk + tt * D + cq * DPL);
+#pragma unroll
+          for (int v = 0; v < DPL / 8; ++v) {
+            const uint4 w = kr[v];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[e]));
+              partial = fmaf(qf[8 * v + 2 * e], f.x, partial);
+              partial = fmaf(qf[8 * v + 2 * e + 1], f.y, partial);
+            }
+          }
+        }
+        partial += __shfl_xor_sync(0xffffffffu, partial, 1);
+        partial += __shfl_xor_sync(0xffffffffu, partial, 2);
+        sc[u] = valid ? partial * inv_sqrt_d : -INFINITY;
+        mloc = fmaxf(mloc, sc[u]);
+      }
+      const float m_c = warp_max(mloc);
+      if (m_c != -INFINITY) {
+        const float m_new = fmaxf(m_run, m_c);
+        const float alpha = m_run == -INFINITY ? 0.f : __expf(m_run - m_new);
+        float pr[TW / 8];
+        float my_s = 0.f;
+#pragma unroll
+        for (int u = 0; u < TW / 8; ++u) {
+          pr[u] = sc[u] == -INFINITY ? 0.f : __expf(sc[u] - m_new);
+          if (cq == 0) my_s += pr[u];
+        }
+        const float s_c = warp_sum(my_s);
+        float part_v[DPV];
+#pragma unroll
+        for (int e = 0; e < DPV; ++e) part_v[e] = 0.f;
+#pragma unroll
+        for (int u = 0; u < TW / 8; ++u) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float p = __shfl_sync(0xffffffffu, pr[u], 4 * k);
+            const int tt = wt0 + u * 8 + k;
+            if (tt < nt) {
+              const __half* vr = sv + tt * D + lane * DPV;
+#pragma unroll
+              for (int e = 0; e < DPV; e += 2) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(vr + e));
+                part_v[e] = fmaf(p, f.x, part_v[e]);
+                part_v[e + 1] = fmaf(p, f.y, part_v[e + 1]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < DPV; ++e) acc[e] = acc[e] * alpha + part_v[e];
+        l_run = l_run * alpha + s_c;
+        m_run = m_new;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (lane == 0) {
+      cm[warp] = m_run;
+      cl[warp] = l_run;
+    }
+#pragma unroll
+    for (int e = 0; e < DPV; ++e) cacc[warp][lane * DPV + e] = acc[e];
+  }
+  __syncthreads();
+  merge_and_store<D>(cm, cl, cacc, out, ldo, i, j, hr, z, part, ctr, &last_flag);
+}
+
+template <int D>
+cudaError_t launch_f16(const __half* q, int ldq, const KvView& kv, int b, int heads, int len, __half* out, int ldo,
+                       int splits, float* part, int* ctr, cudaStream_t s) {
+  using L = F16Stage<D>;
+  static cudaError_t attr = cudaFuncSetAttribute(attn_decode_f16_kernel<D>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, L::stages * L::bytes);
+  if (attr != cudaSuccess) return attr;
+  int span = (len + splits - 1) / splits;
+  span = (span + L::T - 1) / L::T * L::T;
+  const int S = (len + span - 1) / span;
+  dim3 grid(heads, b, S);
+  attn_decode_f16_kernel<D><<<grid, kQ4Threads, L::stages * L::bytes, s>>>(
+      q, ldq, kv, heads, len, out, ldo, 1.0f / sqrtf(static_cast<float>(D)), span, part, ctr,
+      runtime().wait_limit_ns, runtime().err);
   return launched();
 }
 
@@ -634,12 +656,12 @@ cudaError_t launch_attn_decode(const __half* q, int ldq, const KvView& kv, int b
                                int kv_bits, int len, __half* out, int ldo, float* part, int* ctr,
                                cudaStream_t s) {
   if (b == 0) return cudaSuccess;
-  const int splits = (part != nullptr && ctr != nullptr && kv_bits == 4) ? attn_decode_splits(b, heads, len) : 1;
+  const int splits = (part != nullptr && ctr != nullptr) ? attn_decode_splits(b, heads, len) : 1;
   if (d == 128)
     return kv_bits == 4 ? launch_q4<128>(q, ldq, kv, b, heads, len, out, ldo, splits, part, ctr, s)
-                        : launch_one<128, 16>(q, ldq, kv, b, heads, len, out, ldo, s);
+                        : launch_f16<128>(q, ldq, kv, b, heads, len, out, ldo, splits, part, ctr, s);
   return kv_bits == 4 ? launch_q4<64>(q, ldq, kv, b, heads, len, out, ldo, splits, part, ctr, s)
-                      : launch_one<64, 16>(q, ldq, kv, b, heads, len, out, ldo, s);
+                      : launch_f16<64>(q, ldq, kv, b, heads, len, out, ldo, splits, part, ctr, s);
 }
 
 }  // namespace flexq

@@ -532,7 +532,6 @@ flexq_status flexq_linear(const void* x_dev, int ldx, const void* w_dev, int w_b
   FQ_CHECK(x_dev && w_dev && y_dev, "NULL pointer");
   FQ_CHECK(ldx >= k && ldx % 8 == 0 && aligned16(x_dev), "x needs ldx >= k, ldx %% 8 == 0, 16-byte alignment");
   FQ_CHECK(aligned16(w_dev), "w must be 16-byte aligned");
-  FQ_CHECK(w_bits == 16 || true, "");
   FQ_CHECK(ldy >= n, "ldy must be >= n");
   FQ_CHECK(!(epilogue & EPI_BIAS) || bias_dev, "bias flag without bias");
   FQ_CHECK(!(epilogue & EPI_RESIDUAL) || (residual_dev && ld_res >= n), "residual flag without residual");

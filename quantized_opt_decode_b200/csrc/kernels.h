@@ -125,8 +125,8 @@ size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits)
 cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
 
 // attention
-// Decode attention.  With part/ctr (a 4-bit cache only): when b * heads
-// CTAs cannot fill the GPU, each (sequence, head) is split over several CTAs
+// Decode attention.  With part/ctr: when b * heads CTAs cannot fill the
+// GPU, each (sequence, head) is split over several CTAs
 // along the cache, partial results go to `part`
 // (attn_decode_partial_bytes) and the last split of each merges them;
 // ctr = b * heads ints, zero on entry and left zero.

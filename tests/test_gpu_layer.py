@@ -309,3 +309,31 @@ def test_offloaded_weights_match_resident(gbs):
     with pytest.raises(fq.FlexqError) as ei:
         fq.flexq_generate_offload(res.struct, slots, 2 * slot, copy, prompts, b, s, n, gbs, out_o, ws, ws_n)
     assert ei.value.status == 1 and "page-locked" in str(ei.value)
+
+
+def test_layer_decode_long_fp16_cache():
+    """The fp16-cache decode attention over a long cache split across CTAs
+    (b * heads = 4 pairs), against the oracle's decode on the same fp16 rows."""
+    p = _preset("tiny16", h=256, heads=4, ffn=1024)
+    h, b, length = p["h"], 1, 900
+    cfg = opt.Config.from_preset(p, ln1_f16=True)
+    seed = synth.config_seed(p)
+    W = opt.effective_layer(cfg, opt.raw_layer(cfg, seed, 0))
+    dm = DeviceModel(p, b=b, max_len=length + 2, layers=1)
+    rng = np.random.default_rng(91)
+    rows = rng.standard_normal((b * length, 2 * h)).astype(np.float16)
+    t = rng.standard_normal((b, h)).astype(np.float16)
+    rd = to_dev(rows)
+    kv = dm.kv[0].struct
+    fq.flexq_kv_append(dm.cfg, kv, rd[:, :h], rd[:, h:], 2 * h, b, 0, length)
+    ws_n = fq.flexq_layer_workspace(dm.cfg, b, 1)
+    ws = workspace(ws_n)
+    td = to_dev(t)
+    t2 = torch.empty_like(td)
+    fq.flexq_layer_decode(dm.cfg, dm.layers[0].struct, td, t2, kv, b, length, ws, ws_n)
+    fq.flexq_device_status()
+    cache = opt.KVCache(cfg, b, length + 2, 16)
+    cache.write("k", rows[:, :h].reshape(b, length, h), 0)
+    cache.write("v", rows[:, h:].reshape(b, length, h), 0)
+    ref = opt.layer_decode(cfg, W, t.astype(np.float64), cache, length)
+    _check_out(to_host(t2), ref, t)
