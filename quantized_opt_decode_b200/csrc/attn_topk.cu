@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "quant_common.cuh"
 
 namespace flexq {
 namespace {
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
                                                                   int heads, int len, int kk,
                                                                   __half* __restrict__ out, int ldo,
                                                                   int32_t* __restrict__ idx_out,
-                                                                  float inv_sqrt_d) {
+                                                                  float inv_sqrt_d, AppendRow app) {
   constexpr int G = D / 64;
   constexpr int DPL = D / 4;
   constexpr int NW = DPL / 8;
@@ -103,6 +104,12 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
   const __half2* km = static_cast<const __half2*>(kv.k_meta) + hr * kv.max_len * G;
   const __half2* vm = static_cast<const __half2*>(kv.v_meta) + hr * kv.max_len * G;
   const uint32_t* vw = static_cast<const uint32_t*>(kv.v) + hr * (kv_pad_len(kv.max_len) / 8) * D;
+
+  // decode: this token's K/V rows enter the cache before the scores read it
+  if (app.pos >= 0) {
+    if (warp == 0) append_row_q4<D>(app, kv, i, j, heads);
+    __syncthreads();
+  }
 
   // ---- scores (all keys)
   const int cq = lane & 3, g = (cq * DPL) / 64;
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
 
 template <int D>
 cudaError_t launch_topk(const __half* q, int ldq, const KvView& kv, int b, int heads, int len, int kk, __half* out,
-                        int ldo, int32_t* idx, cudaStream_t s) {
+                        int ldo, int32_t* idx, const AppendRow& app, cudaStream_t s) {
   const size_t smem = static_cast<size_t>((len + 3) & ~3) * sizeof(float) + static_cast<size_t>((len + 15) & ~15);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(attn_topk_q4_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -326,17 +333,17 @@ cudaError_t launch_topk(const __half* q, int ldq, const KvView& kv, int b, int h
   }
   dim3 grid(heads, b);
   attn_topk_q4_kernel<D><<<grid, kTkThreads, smem, s>>>(q, ldq, kv, heads, len, kk, out, ldo, idx,
-                                                        1.0f / sqrtf(static_cast<float>(D)));
+                                                        1.0f / sqrtf(static_cast<float>(D)), app);
   return launched();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_topk(const __half* q, int ldq, const KvView& kv, int b, int heads, int d, int len, int kk,
-                             __half* out, int ldo, int32_t* idx, cudaStream_t s) {
+                             __half* out, int ldo, int32_t* idx, const AppendRow& app, cudaStream_t s) {
   if (b == 0) return cudaSuccess;
-  return d == 128 ? launch_topk<128>(q, ldq, kv, b, heads, len, kk, out, ldo, idx, s)
-                  : launch_topk<64>(q, ldq, kv, b, heads, len, kk, out, ldo, idx, s);
+  return d == 128 ? launch_topk<128>(q, ldq, kv, b, heads, len, kk, out, ldo, idx, app, s)
+                  : launch_topk<64>(q, ldq, kv, b, heads, len, kk, out, ldo, idx, app, s);
 }
 
 }  // namespace flexq

@@ -246,14 +246,15 @@ flexq_status run_linear(const __half* x, int ldx, const void* w, int w_bits, int
 }
 
 // Decode attention of a layer step: dense, or top-k sparse when the config
-// asks for it.
+// asks for it; with app.pos >= 0 it first appends the token's K/V rows to a
+// 4-bit cache.
 cudaError_t decode_attention(const flexq_config* c, const __half* q, int ldq, const KvView& kvv, int b, int len,
-                             __half* out, int ldo, float* part, int* ctr, cudaStream_t s) {
+                             __half* out, int ldo, float* part, int* ctr, const AppendRow& app, cudaStream_t s) {
   const int d = c->h / c->heads;
   if (c->attn_topk_permille > 0)
     return launch_attn_topk(q, ldq, kvv, b, c->heads, d, len, topk_count(len, c->attn_topk_permille), out, ldo,
-                            nullptr, s);
-  return launch_attn_decode(q, ldq, kvv, b, c->heads, d, c->kv_bits, len, out, ldo, part, ctr, s);
+                            nullptr, app, s);
+  return launch_attn_decode(q, ldq, kvv, b, c->heads, d, c->kv_bits, len, out, ldo, part, ctr, app, s);
 }
 
 // The fused decode step takes at most one token tile of sequences.
@@ -261,12 +262,13 @@ bool decode_fusable(int b) { return b >= 1 && b <= kFuseMaxRows; }
 
 // Decode step of one layer for b sequences, fused ([WT] "P/D阶段计算",
 // decoding phase): u_in = LN1(t) computed by the caller (the previous
-// layer's FC2 or the embedding); the QKV projection appends this token's K/V
-// to cache slot pos in its epilogue; attention reads slots 0..pos; the
-// output projection adds the residual and LayerNorms its rows (LN2) after a
-// grid barrier; FC1 + GELU; FC2 adds the residual and, when ln_next_g is
-// set, LayerNorms its rows into u_out (the next layer's LN1 or the final
-// LN).  w.ctr must be zero (it is left zero).
+// layer's FC2 or the embedding); the QKV projection stores this token's K/V
+// straight into an fp16 cache slot pos, or the decode attention quantizes
+// them into a 4-bit cache slot pos before it reads slots 0..pos; the output
+// projection adds the residual and LayerNorms its rows (LN2) after a grid
+// barrier; FC1 + GELU; FC2 adds the residual and, when ln_next_g is set,
+// LayerNorms its rows into u_out (the next layer's LN1 or the final LN).
+// w.ctr must be zero (it is left zero).
 flexq_status decode_fused(const flexq_config* c, const flexq_layer* L, const __half* t, const __half* u_in,
                           __half* y, __half* u_out, const void* ln_next_g, const void* ln_next_b,
                           const flexq_kv* kv, int seq0, int b, int pos, const LayerWs& w, cudaStream_t s) {
@@ -274,25 +276,30 @@ flexq_status decode_fused(const flexq_config* c, const flexq_layer* L, const __h
   const KvView kvv = view_of(c, kv, seq0);
   int* tile_ctr = w.tile_ctr;
   KvFuse kf{};
-  kf.k_codes = static_cast<uint8_t*>(kvv.k);
-  kf.v_words = static_cast<uint32_t*>(kvv.v);
-  kf.k_meta = static_cast<__half2*>(kvv.k_meta);
-  kf.v_meta = static_cast<__half2*>(kvv.v_meta);
-  kf.h = h;
-  kf.heads = c->heads;
-  kf.d = d;
-  kf.max_len = kvv.max_len;
-  kf.pos = pos;
-  kf.bits = c->kv_bits;
+  AppendRow app = kNoAppend;
+  if (c->kv_bits == 16) {
+    kf.k = static_cast<__half*>(kvv.k);
+    kf.v = static_cast<__half*>(kvv.v);
+    kf.h = h;
+    kf.heads = c->heads;
+    kf.d = d;
+    kf.max_len = kvv.max_len;
+    kf.pos = pos;
+  } else {
+    app.k = w.qkv + h;
+    app.v = w.qkv + 2 * h;
+    app.ld = 3 * h;
+    app.pos = pos;
+  }
   {
     ProfScope ps(FLEXQ_K_QKV, s);
     FQ_TRY(run_linear(u_in, h, L->w_qkv, c->w_bits, b, 3 * h, h, static_cast<const __half*>(L->b_qkv), nullptr, 0,
-                      EPI_BIAS, w.qkv, 3 * h, w.acc, w.acc_bytes, s, "QKV projection with KV append", &kf, nullptr,
-                      tile_ctr));
+                      EPI_BIAS, w.qkv, 3 * h, w.acc, w.acc_bytes, s, "QKV projection",
+                      c->kv_bits == 16 ? &kf : nullptr, nullptr, tile_ctr));
   }
   {
     ProfScope ps(FLEXQ_K_ATTN_DECODE, s);
-    FQ_CUDA(decode_attention(c, w.qkv, 3 * h, kvv, b, pos + 1, w.o, h, w.attn_part, w.attn_ctr, s),
+    FQ_CUDA(decode_attention(c, w.qkv, 3 * h, kvv, b, pos + 1, w.o, h, w.attn_part, w.attn_ctr, app, s),
             "decode attention");
   }
   LnFuse ln2{};
@@ -356,7 +363,8 @@ flexq_status layer_step(const flexq_config* c, const flexq_layer* L, const __hal
     FQ_CUDA(launch_attn_prefill(w.qkv, 3 * h, b, ntok, c->heads, d, w.u, h, s), "prefill attention");
   } else {
     ProfScope ps(FLEXQ_K_ATTN_DECODE, s);
-    FQ_CUDA(decode_attention(c, w.qkv, 3 * h, kvv, b, pos + 1, w.u, h, nullptr, nullptr, s), "decode attention");
+    FQ_CUDA(decode_attention(c, w.qkv, 3 * h, kvv, b, pos + 1, w.u, h, nullptr, nullptr, kNoAppend, s),
+            "decode attention");
   }
   {
     ProfScope ps(FLEXQ_K_OUT_PROJ, s);
@@ -612,7 +620,7 @@ flexq_status flexq_attention_decode(const flexq_config* cfg, const flexq_kv* kv,
   FQ_CHECK(ldq >= cfg->h && ldo >= cfg->h && ldq % 8 == 0 && ldo % 8 == 0, "bad row strides");
   FQ_CUDA(launch_attn_decode(static_cast<const __half*>(q_dev), ldq, view_of(cfg, kv, 0), b, cfg->heads,
                              cfg->h / cfg->heads, cfg->kv_bits, len, static_cast<__half*>(out_dev), ldo, nullptr,
-                             nullptr, as_stream(stream)),
+                             nullptr, kNoAppend, as_stream(stream)),
           "decode attention");
   return FLEXQ_OK;
 }
@@ -629,7 +637,8 @@ flexq_status flexq_attention_decode_topk(const flexq_config* cfg, const flexq_kv
   FQ_CHECK(q_dev && out_dev, "NULL pointer");
   FQ_CHECK(ldq >= cfg->h && ldo >= cfg->h && ldq % 8 == 0 && ldo % 8 == 0, "bad row strides");
   FQ_CUDA(launch_attn_topk(static_cast<const __half*>(q_dev), ldq, view_of(cfg, kv, 0), b, cfg->heads,
-                           cfg->h / cfg->heads, len, k, static_cast<__half*>(out_dev), ldo, idx_dev, as_stream(stream)),
+                           cfg->h / cfg->heads, len, k, static_cast<__half*>(out_dev), ldo, idx_dev, kNoAppend,
+                           as_stream(stream)),
           "top-k decode attention");
   return FLEXQ_OK;
 }

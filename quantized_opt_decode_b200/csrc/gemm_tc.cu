@@ -46,7 +46,6 @@
 
 #include "common.cuh"
 #include "kernels.h"
-#include "quant_common.cuh"
 
 namespace flexq {
 namespace {
@@ -56,13 +55,11 @@ constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
 constexpr int kATileBytes = 128 * 64 * 2;
-constexpr int kRawStageBytes = (kTileBytes + 1023) / 1024 * 1024;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
 constexpr int kMaxBarriers = 56;     // mbarriers fit in the first 448 bytes of that region
 constexpr int kEpiStageBytes = 4 * 16 * 33 * 4;  // per epilogue warp: 16 tokens x 33 floats
-constexpr int kKvStageBytes = 16 * 128 * 2;      // fp16 K/V rows of 16 tokens x 128 features
-constexpr int kMaxLoadStages = 16;
+constexpr int kMaxWStages = 16;
 constexpr int kMinItersPerCta = 8;
 constexpr int kMaxContrib = 64;
 constexpr int kDecodeMaxTok = 160;
@@ -84,8 +81,8 @@ struct GemmParams {
   int m, n, k;
   int tok_tile;
   int kb_real;  // 64-wide k-blocks of K
-  int load_stages, a_stages;
-  uint32_t load_stage_bytes;
+  int w_stages, b_stages, a_stages;     // ring depths: weights, activations, dequantized A
+  uint32_t w_slot_bytes, b_slot_bytes;
   uint32_t acc_cols;    // TMEM columns between the two accumulator buffers
   uint32_t tmem_alloc;  // columns allocated (power of two)
   Sched sc;
@@ -101,7 +98,7 @@ struct GemmParams {
   int* counters;    // [tiles][2]: contributors arrived, partials published
   uint64_t wait_ns;
   uint32_t* err;
-  int kv_on;        // decode QKV: K/V tiles go to the 4-bit cache
+  int kv_on;        // decode QKV: K/V tiles go to the fp16 cache
   KvFuse kv;
   int ln_on;        // decode out-proj / FC2: LayerNorm of the rows after a grid barrier
   LnFuse ln;
@@ -306,7 +303,6 @@ struct Ctl {
   volatile int* fin_me;
   int* fin_slots;  // [kMaxContrib]
   float* stage;    // [4][16][33]
-  __half* kvst;    // [16][128] fp16 K/V rows of the chunk being quantized
 };
 
 __device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
@@ -320,68 +316,7 @@ __device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
   c.fin_me = c.abort_flag + 3;
   c.fin_slots = reinterpret_cast<int*>(region + kBarrierBytes / 2);
   c.stage = reinterpret_cast<float*>(region + kBarrierBytes);
-  c.kvst = reinterpret_cast<__half*>(region + kBarrierBytes + kEpiStageBytes);
   return c;
-}
-
-// Quantizes the staged fp16 K/V rows of one 16-token chunk into the cache:
-// thread et (< 64, two whole warps) and its neighbour et ^ 1 own one
-// 64-feature group of one token, exactly as the standalone append kernels
-// split a row ("FlexGen研究学术报告" section 三(C): groups of 64 along the
-// head dimension, fp16 min/scale).  K: canonical codes of slot pos; V: the
-// token's nibble in each token-interleaved word (one writer per word, since
-// a decode step appends a single token per sequence).
-__device__ __forceinline__ void kv_quantize_chunk(const GemmParams& p, const __half* kvst, int tokbase,
-                                                  int n_tile, int et) {
-  const int jq = et >> 2, gq = (et >> 1) & 1, half_id = et & 1;
-  const uint4* src = reinterpret_cast<const uint4*>(kvst + jq * 128 + gq * 64 + half_id * 32);
-  float v[32];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const uint4 w = src[u];
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(u32_as_h2(ww[e]));
-      v[8 * u + 2 * e] = f.x;
-      v[8 * u + 2 * e + 1] = f.y;
-    }
-  }
-  uint32_t q[32];
-  __half m16, s16;
-  q64_lane_pair(v, q, m16, s16);
-  const int tok = tokbase + jq;
-  if (tok >= p.m) return;
-  const KvFuse& kv = p.kv;
-  const int col = n_tile * 128 + gq * 64;
-  const bool is_v = col >= 2 * kv.h;
-  const int cc = col - (is_v ? 2 * kv.h : kv.h);
-  const int j = cc / kv.d, gd = (cc % kv.d) / 64;
-  const size_t hr = static_cast<size_t>(tok) * kv.heads + j;
-  const size_t slot = hr * kv.max_len + kv.pos;
-  if (!is_v) {
-    const uint4 out = make_uint4(pack_canonical(q), pack_canonical(q + 8), pack_canonical(q + 16),
-                                 pack_canonical(q + 24));
-    *reinterpret_cast<uint4*>(kv.k_codes + slot * (kv.d / 2) + gd * 32 + half_id * 16) = out;
-    if (half_id == 0) kv.k_meta[slot * (kv.d / 64) + gd] = __halves2half2(m16, s16);
-  } else {
-    uint4* w4 = reinterpret_cast<uint4*>(kv.v_words + (hr * (kv_pad_len(kv.max_len) / 8) + kv.pos / 8) * kv.d +
-                                         gd * 64 + half_id * 32);
-    const int sh = 4 * (kv.pos & 7);
-    const uint32_t clear = ~(0xFu << sh);
-    uint4 cur[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) cur[u] = w4[u];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      cur[u].x = (cur[u].x & clear) | (q[4 * u] << sh);
-      cur[u].y = (cur[u].y & clear) | (q[4 * u + 1] << sh);
-      cur[u].z = (cur[u].z & clear) | (q[4 * u + 2] << sh);
-      cur[u].w = (cur[u].w & clear) | (q[4 * u + 3] << sh);
-      w4[u] = cur[u];
-    }
-    if (half_id == 0) kv.v_meta[slot * (kv.d / 64) + gd] = __halves2half2(m16, s16);
-  }
 }
 
 // Bounded wait until a global counter reaches `target` (the other
@@ -427,7 +362,7 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
     const uint32_t tbase =
         tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + (static_cast<uint32_t>(qd * 32) << 16);
     const int f_out = n_tile * 128 + qd * 32 + hf * 16;  // features this lane finishes
-    // decode QKV with the cache fused: the K and V tiles are quantized, not stored
+    // decode QKV with an fp16 cache: the K and V tiles go to the cache slot
     const bool kv_tile = p.kv_on && n_tile * 128 >= p.kv.h;
     // Split tile: count in; the last to arrive finishes the tile.
     int ns = 1, me = 0;
@@ -540,34 +475,20 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       __syncwarp();
       const int tok = tok0 + c0 + jt;
       if (kv_tile) {
-        // the chunk's fp16 rows (+ bias, the values the cache receives)
-        uint32_t packed[8];
+        // this lane's 16 features of its token (+ bias) go to slot pos
+        if (tok < p.m) {
+          uint32_t packed[8];
 #pragma unroll
-        for (int u = 0; u < 16; u += 2)
-          packed[u / 2] = h2_as_u32(__floats2half2_rn(stg[jt * 33 + hf * 16 + u] + bv[u],
-                                                      stg[jt * 33 + hf * 16 + u + 1] + bv[u + 1]));
-        if (p.kv.bits == 16) {
-          // fp16 cache: this lane's 16 features of its token go to slot pos
-          if (tok < p.m) {
-            const bool is_v = f_out >= 2 * p.kv.h;
-            const int cc = f_out - (is_v ? 2 * p.kv.h : p.kv.h);
-            __half* base = reinterpret_cast<__half*>(is_v ? static_cast<void*>(p.kv.v_words)
-                                                          : static_cast<void*>(p.kv.k_codes));
-            uint4* dst = reinterpret_cast<uint4*>(
-                base + ((static_cast<size_t>(tok) * p.kv.heads + cc / p.kv.d) * p.kv.max_len + p.kv.pos) * p.kv.d +
-                cc % p.kv.d);
-            dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          }
-        } else {
-          // 4-bit cache: stage in shared memory; two warps then quantize
-          // whole 64-feature groups
-          uint4* dst = reinterpret_cast<uint4*>(c.kvst + jt * 128 + qd * 32 + hf * 16);
+          for (int u = 0; u < 16; u += 2)
+            packed[u / 2] = h2_as_u32(__floats2half2_rn(stg[jt * 33 + hf * 16 + u] + bv[u],
+                                                        stg[jt * 33 + hf * 16 + u + 1] + bv[u + 1]));
+          const bool is_v = f_out >= 2 * p.kv.h;
+          const int cc = f_out - (is_v ? 2 * p.kv.h : p.kv.h);
+          uint4* dst = reinterpret_cast<uint4*>(
+              (is_v ? p.kv.v : p.kv.k) +
+              ((static_cast<size_t>(tok) * p.kv.heads + cc / p.kv.d) * p.kv.max_len + p.kv.pos) * p.kv.d + cc % p.kv.d);
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-          epi_bar();
-          if (et < 64) kv_quantize_chunk(p, c.kvst, tok0 + c0, n_tile, et);
-          epi_bar();
         }
       } else if (tok < p.m && f_out < p.n) {
         float o[16];
@@ -715,10 +636,38 @@ __device__ __forceinline__ void teardown(const GemmParams& p, const Ctl& c, uint
 }
 
 // ---------------------------------------------------------------------------
-// general kernel: A tiles in shared memory, one MMA-issuing thread
+// the kernel: A tiles in shared memory, one MMA-issuing thread
 // ---------------------------------------------------------------------------
-// KS: 64-wide k-blocks per pipeline stage (k-step); two halve the mbarrier
-// hand-offs per tile, which bound decode-sized tiles.
+// Walks a CTA's k-steps in order across its segments.
+struct StepCursor {
+  int q = 0, ks = 0;
+  Seg g;
+  bool valid = false;
+  __device__ __forceinline__ void start(const Sched& sc, int cta) {
+    q = 0;
+    valid = get_seg(sc, cta, 0, g);
+    ks = valid ? g.kb0 : 0;
+  }
+  __device__ __forceinline__ void next(const Sched& sc, int cta) {
+    if (++ks < g.kb1) return;
+    ++q;
+    valid = get_seg(sc, cta, q, g);
+    if (valid) ks = g.kb0;
+  }
+};
+
+// KS: 64-wide k-blocks per k-step (two halve the mbarrier hand-offs per
+// tile, which bound decode-sized tiles).  Three rings in shared memory:
+//   W  weight chunks (4-bit: the packed codes + (min, scale); fp16: TMA tiles
+//      that are the MMA's A operand directly), filled by the producer far
+//      ahead of use: the weights stream from HBM, so the bytes this SM keeps
+//      in flight set the rate at which it receives them;
+//   B  activation boxes (from L2, a short ring);
+//   A  dequantized fp16 tiles (4-bit only), written by the dequantizing warps.
+// The producer issues in the order W(0 .. SW-1), then B(i), W(i + SW) for
+// i = 0, 1, ..: B(i) waits for the MMA of step i - SB, W(i + SW) for the
+// dequantizing warps to have read step i (they release a W slot as soon as
+// its codes are in registers), so the weight ring runs a whole ring ahead.
 template <bool kW4, int KS>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
@@ -726,14 +675,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const int SL = p.load_stages, SA = p.a_stages;
+  const int SW = p.w_stages, SB = p.b_stages, SA = p.a_stages;
   constexpr uint32_t a_slot_bytes = KS * kATileBytes;
-  uint8_t* a_ring = smem;                       // SA x KS fp16 A tiles (4-bit weights only)
-  uint8_t* l_ring = smem + SA * a_slot_bytes;   // SL x load_stage_bytes
-  uint8_t* region = l_ring + SL * p.load_stage_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(region);
-  uint64_t* empty = full + SL;
-  uint64_t* afull = empty + SL;
+  uint8_t* a_ring = smem;                                // SA x KS fp16 A tiles (4-bit weights only)
+  uint8_t* w_ring = a_ring + SA * a_slot_bytes;          // SW x w_slot_bytes
+  uint8_t* b_ring = w_ring + SW * p.w_slot_bytes;        // SB x b_slot_bytes
+  uint8_t* region = b_ring + SB * p.b_slot_bytes;
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(region);
+  uint64_t* wempty = wfull + SW;
+  uint64_t* bfull = wempty + SW;
+  uint64_t* bempty = bfull + SB;
+  uint64_t* afull = bempty + SB;
   uint64_t* aempty = afull + SA;
   uint64_t* drained = aempty + SA;
   const Ctl c = make_ctl(region, drained + 1);
@@ -742,14 +694,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
   const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;  // one 64-wide activation box
-  // load slot: 4-bit = [KS activation boxes | KS raw chunks]; fp16 = [KS weight boxes | KS activation boxes]
-  const uint32_t b_off = kW4 ? 0u : static_cast<uint32_t>(KS * kATileBytes);
-  const uint32_t raw_off = KS * b_bytes;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SL; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], kW4 ? kDequantThreads : 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(&bfull[s], 1);
+      mbar_init(&bempty[s], 1);
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(&afull[s], kDequantThreads);
@@ -780,51 +733,74 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!kW4) prefetch_tmap(&tmap_w);
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      const uint32_t tx_bytes =
-          KS * ((kW4 ? static_cast<uint32_t>(kTileBytes) : static_cast<uint32_t>(kATileBytes)) + b_bytes);
-      int i = 0;
-      Ring rl;
-      Seg g;
+      const uint32_t w_tx = KS * (kW4 ? static_cast<uint32_t>(kTileBytes) : static_cast<uint32_t>(kATileBytes));
+      const uint32_t b_tx = KS * b_bytes;
+      StepCursor wc, bc;
+      wc.start(sc, cta);
+      bc.start(sc, cta);
+      Ring rw, rb;
+      int nw = 0, nb = 0;
       bool stop = false;
-      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-        const int n_tile = g.tile % sc.n_tiles;
-        const int t_row = (g.tile / sc.n_tiles) * p.tok_tile;
-        const uint8_t* wsrc = p.wq + (static_cast<size_t>(n_tile) * p.kb_real + g.kb0 * KS) * kTileBytes;
-        for (int ks = g.kb0; ks < g.kb1; ++ks, ++i, rl.next(SL), wsrc += KS * kTileBytes) {
-          const int s = rl.s;
-          if (!mbar_wait(&empty[s], rl.ph ^ 1u, p.wait_ns)) {
-            set_error(p.err, DEV_TIMEOUT_PRODUCER);
-            *c.abort_flag = 1;
-          }
-          if (*c.abort_flag) {
-            stop = true;
-            break;
-          }
-          uint8_t* st = l_ring + s * p.load_stage_bytes;
-          mbar_arrive_expect_tx(&full[s], tx_bytes);
-          if (kW4) bulk_load(st + raw_off, wsrc, KS * kTileBytes, &full[s], pol_w);
-#pragma unroll
-          for (int u = 0; u < KS; ++u) {
-            const int kx = (ks * KS + u) * 64;
-            if (!kW4) tma_load_2d(st + u * kATileBytes, &tmap_w, &full[s], kx, n_tile * 128, pol_w);
-            tma_load_2d(st + b_off + u * b_bytes, &tmap_x, &full[s], kx, t_row, pol_x);
-          }
+      auto slot_free = [&](uint64_t* bar, const Ring& r) {
+        if (!mbar_wait(bar, r.ph ^ 1u, p.wait_ns)) {
+          set_error(p.err, DEV_TIMEOUT_PRODUCER);
+          *c.abort_flag = 1;
         }
+        return *c.abort_flag == 0;
+      };
+      auto issue_w = [&]() {
+        if (!slot_free(&wempty[rw.s], rw)) return false;
+        const int n_tile = wc.g.tile % sc.n_tiles;
+        uint8_t* dst = w_ring + rw.s * p.w_slot_bytes;
+        mbar_arrive_expect_tx(&wfull[rw.s], w_tx);
+        if (kW4) {
+          bulk_load(dst, p.wq + (static_cast<size_t>(n_tile) * p.kb_real + wc.ks * KS) * kTileBytes, KS * kTileBytes,
+                    &wfull[rw.s], pol_w);
+        } else {
+#pragma unroll
+          for (int u = 0; u < KS; ++u)
+            tma_load_2d(dst + u * kATileBytes, &tmap_w, &wfull[rw.s], (wc.ks * KS + u) * 64, n_tile * 128, pol_w);
+        }
+        rw.next(SW);
+        ++nw;
+        wc.next(sc, cta);
+        return true;
+      };
+      auto issue_b = [&]() {
+        if (!slot_free(&bempty[rb.s], rb)) return false;
+        const int t_row = (bc.g.tile / sc.n_tiles) * p.tok_tile;
+        uint8_t* dst = b_ring + rb.s * p.b_slot_bytes;
+        mbar_arrive_expect_tx(&bfull[rb.s], b_tx);
+#pragma unroll
+        for (int u = 0; u < KS; ++u)
+          tma_load_2d(dst + u * b_bytes, &tmap_x, &bfull[rb.s], (bc.ks * KS + u) * 64, t_row, pol_x);
+        rb.next(SB);
+        ++nb;
+        bc.next(sc, cta);
+        return true;
+      };
+      while (!stop && wc.valid && nw < SW) stop = !issue_w();
+      while (!stop && bc.valid) {
+        stop = !issue_b();
+        if (!stop && wc.valid) stop = !issue_w();
       }
       // Never leave the CTA with bulk copies still landing in its shared memory.
-      for (int j = max(0, i - SL); j < i; ++j)
-        mbar_wait(&full[j % SL], static_cast<uint32_t>(j / SL) & 1u, drain_ns(p.wait_ns));
+      for (int j = max(0, nw - SW); j < nw; ++j)
+        mbar_wait(&wfull[j % SW], static_cast<uint32_t>(j / SW) & 1u, drain_ns(p.wait_ns));
+      for (int j = max(0, nb - SB); j < nb; ++j)
+        mbar_wait(&bfull[j % SB], static_cast<uint32_t>(j / SB) & 1u, drain_ns(p.wait_ns));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
       // descriptors of slot 0; a slot is reached by adding its byte offset >> 4
-      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(kW4 ? a_ring : l_ring));
-      const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(l_ring + b_off));
-      const uint32_t a_step = (kW4 ? a_slot_bytes : p.load_stage_bytes) >> 4;
-      const uint32_t l_step = p.load_stage_bytes >> 4;
-      Ring rl, ra;
+      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(kW4 ? a_ring : w_ring));
+      const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(b_ring));
+      const uint32_t a_step = (kW4 ? a_slot_bytes : p.w_slot_bytes) >> 4;
+      const uint32_t b_step = p.b_slot_bytes >> 4;
+      const int SAx = kW4 ? SA : SW;  // the ring the A operand sits in
+      Ring rb, ra;
       Seg g;
       bool stop = false;
       for (int q = 0; get_seg(sc, cta, q, g); ++q) {
@@ -838,10 +814,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*c.abort_flag) stop = true;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols;
-        for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, rl.next(SL), ra.next(SA)) {
-          const int s = rl.s;
-          const int sa = kW4 ? ra.s : 0;
-          const bool ok = kW4 ? mbar_wait(&afull[sa], ra.ph, p.wait_ns) : mbar_wait(&full[s], rl.ph, p.wait_ns);
+        for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, rb.next(SB), ra.next(SAx)) {
+          bool ok = kW4 ? mbar_wait(&afull[ra.s], ra.ph, p.wait_ns) : mbar_wait(&wfull[ra.s], ra.ph, p.wait_ns);
+          ok = ok && mbar_wait(&bfull[rb.s], rb.ph, p.wait_ns);
           if (!ok) {
             set_error(p.err, DEV_TIMEOUT_MMA);
             *c.abort_flag = 1;
@@ -850,16 +825,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          const uint64_t adesc = adesc0 + static_cast<uint64_t>((kW4 ? sa : s) * a_step);
-          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * l_step);
+          const uint64_t adesc = adesc0 + static_cast<uint64_t>(ra.s * a_step);
+          const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(rb.s * b_step);
 #pragma unroll
           for (int u = 0; u < KS; ++u)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_f16_ss(d_tmem, adesc + u * (kATileBytes >> 4) + 2 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk, idesc,
                          (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&empty[s]);
-          if (kW4) mma_commit(&aempty[sa]);
+          mma_commit(&bempty[rb.s]);
+          mma_commit(kW4 ? &aempty[ra.s] : &wempty[ra.s]);
         }
         // Every segment ends with a commit, also after an abort, so the
         // epilogue never waits on a barrier nobody signals.
@@ -875,15 +850,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ct = threadIdx.x - 64;
       const int row = ct >> 1;
       const int hf = ct & 1;
-      Ring rl, ra;
+      Ring rw, ra;
       Seg g;
       bool stop = false;
       for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
-        for (int ks = g.kb0; ks < g.kb1; ++ks, rl.next(SL), ra.next(SA)) {
-          const int s = rl.s;
-          const int sa = ra.s;
-          bool ok = mbar_wait(&full[s], rl.ph, p.wait_ns);
-          ok = ok && mbar_wait(&aempty[sa], ra.ph ^ 1u, p.wait_ns);
+        for (int ks = g.kb0; ks < g.kb1; ++ks, rw.next(SW), ra.next(SA)) {
+          bool ok = mbar_wait(&wfull[rw.s], rw.ph, p.wait_ns);
+          ok = ok && mbar_wait(&aempty[ra.s], ra.ph ^ 1u, p.wait_ns);
           if (!ok) {
             set_error(p.err, DEV_TIMEOUT_CONSUMER);
             *c.abort_flag = 1;
@@ -892,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          const uint8_t* raw = l_ring + s * p.load_stage_bytes + raw_off;
+          const uint8_t* raw = w_ring + rw.s * p.w_slot_bytes;
           uint4 cw[KS];
           __half2 mm[KS];
 #pragma unroll
@@ -900,11 +873,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             cw[u] = *reinterpret_cast<const uint4*>(raw + u * kTileBytes + row * 32 + hf * 16);
             mm[u] = *reinterpret_cast<const __half2*>(raw + u * kTileBytes + kTileCodeBytes + row * 4);
           }
+          // the codes are in registers: the weight slot may be refilled
+          mbar_arrive(&wempty[rw.s]);
 #pragma unroll
           for (int u = 0; u < KS; ++u) {
             const __half2 m2 = __low2half2(mm[u]);
             const __half2 s2 = __high2half2(mm[u]);
-            uint8_t* arow = a_ring + sa * a_slot_bytes + u * kATileBytes + row * 128;
+            uint8_t* arow = a_ring + ra.s * a_slot_bytes + u * kATileBytes + row * 128;
             const uint32_t words[4] = {cw[u].x, cw[u].y, cw[u].z, cw[u].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -913,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           fence_proxy_async_smem();
-          mbar_arrive(&afull[sa]);
+          mbar_arrive(&afull[ra.s]);
         }
       }
     }
@@ -1001,8 +976,8 @@ struct Plan {
   int tok_tile, tok_tiles, n_tiles;
   int ks;       // k-blocks per stage of gemm_tc_kernel
   Sched sc;
-  int load_stages, a_stages;
-  uint32_t load_stage_bytes;
+  int w_stages, b_stages, a_stages;
+  uint32_t w_slot_bytes, b_slot_bytes;
   uint32_t acc_cols, tmem_alloc;
   size_t smem;
   size_t partial_bytes, counter_bytes;
@@ -1065,26 +1040,27 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.partial_bytes = static_cast<size_t>(2) * s.grid * tile_bytes;
   }
   if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * 2 * sizeof(int);
-  const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes - kKvStageBytes;
-  const int b_bytes = P.tok_tile * 128;
-  int a_slot = 0;
+  // Shared memory: the A ring (4-bit), a short activation ring, and as deep a
+  // weight ring as the rest allows (the bytes of weights in flight per SM set
+  // the rate at which they arrive from HBM).  Three activation slots when
+  // that still leaves room for at least 8 weight k-steps, else two.
+  const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
   {
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
     P.acc_cols = cols;
     P.tmem_alloc = 2 * cols;
-    if (w_bits == 4) {
-      a_slot = P.ks * kATileBytes;
-      P.a_stages = P.ks == 2 ? 2 : (P.tok_tile > 128 && P.tok_tile != 144 ? 2 : 3);
-      P.load_stage_bytes = static_cast<uint32_t>(P.ks * b_bytes + round_up(P.ks * kTileBytes, 1024));
-    } else {
-      P.a_stages = 0;
-      P.load_stage_bytes = static_cast<uint32_t>(kATileBytes + b_bytes);
-    }
   }
-  P.load_stages = min(kMaxLoadStages, (budget - P.a_stages * a_slot) / static_cast<int>(P.load_stage_bytes));
-  P.smem = static_cast<size_t>(P.a_stages) * a_slot + static_cast<size_t>(P.load_stages) * P.load_stage_bytes +
-           1024 + kBarrierBytes + kEpiStageBytes + kKvStageBytes;
+  const int a_slot = w_bits == 4 ? P.ks * kATileBytes : 0;
+  P.a_stages = w_bits == 4 ? 2 : 0;
+  P.w_slot_bytes = static_cast<uint32_t>(w_bits == 4 ? round_up(P.ks * kTileBytes, 1024) : P.ks * kATileBytes);
+  P.b_slot_bytes = static_cast<uint32_t>(P.ks * P.tok_tile * 128);
+  const int rest = budget - P.a_stages * a_slot;
+  const int w_slot = static_cast<int>(P.w_slot_bytes), b_slot = static_cast<int>(P.b_slot_bytes);
+  P.b_stages = rest - 3 * b_slot >= 8 * w_slot ? 3 : 2;
+  P.w_stages = min(kMaxWStages, (rest - P.b_stages * b_slot) / w_slot);
+  P.smem = static_cast<size_t>(P.a_stages) * a_slot + static_cast<size_t>(P.w_stages) * w_slot +
+           static_cast<size_t>(P.b_stages) * b_slot + 1024 + kBarrierBytes + kEpiStageBytes;
   return P;
 }
 
@@ -1146,11 +1122,11 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   if (a.m == 0 || a.n == 0) return cudaSuccess;
   const Plan P = make_plan(a.m, a.n, a.k, a.w_bits, a.force_splits, a.force_tok_tile);
   const bool w4 = a.w_bits == 4;
-  if (P.load_stages < 2) return cudaErrorInvalidValue;
+  if (P.w_stages < 2 || P.b_stages < 2) return cudaErrorInvalidValue;
   // mbarriers the kernel lays out before its control words (make_ctl):
-  // full/empty per load stage, afull/aempty per A slot, the drain barrier,
+  // full/empty per weight and activation slot, afull/aempty per A slot, the drain barrier,
   // accf/acce x 2
-  const int n_bars = 2 * P.load_stages + 2 * P.a_stages + 5;
+  const int n_bars = 2 * (P.w_stages + P.b_stages + P.a_stages) + 5;
   if (n_bars > kMaxBarriers) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
   if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile)) return cudaErrorInvalidValue;
@@ -1166,9 +1142,11 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.k = a.k;
   p.tok_tile = P.tok_tile;
   p.kb_real = a.k / 64;
-  p.load_stages = P.load_stages;
+  p.w_stages = P.w_stages;
+  p.b_stages = P.b_stages;
   p.a_stages = P.a_stages;
-  p.load_stage_bytes = P.load_stage_bytes;
+  p.w_slot_bytes = P.w_slot_bytes;
+  p.b_slot_bytes = P.b_slot_bytes;
   p.acc_cols = P.acc_cols;
   p.tmem_alloc = P.tmem_alloc;
   p.sc = P.sc;
@@ -1202,7 +1180,7 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   if (a.kv != nullptr) {
     // whole 64-feature groups of one head per K/V tile; one token tile
     if (a.m > kFuseMaxRows || P.tok_tiles != 1 || a.n != 3 * a.kv->h || a.kv->h % 128 != 0 ||
-        (a.epi & ~EPI_BIAS) != 0 || (a.kv->bits != 4 && a.kv->bits != 16))
+        (a.epi & ~EPI_BIAS) != 0)
       return cudaErrorInvalidValue;
     p.kv_on = 1;
     p.kv = *a.kv;

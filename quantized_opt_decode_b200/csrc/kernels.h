@@ -79,19 +79,16 @@ enum Epilogue : int {
   EPI_F32_OUT = 8,    // write fp32 (no bias/act/residual allowed)
 };
 // Decode-step fusions of a linear layer (one token per sequence, m rows):
-// KvFuse makes the QKV projection write its K and V columns straight into
-// cache slot `pos` of each of the m sequences (4-bit: quantized, bit-exact
-// with launch_kv_append on the same fp16 rows; 16-bit: the fp16 values)
-// instead of storing them;
+// KvFuse makes the QKV projection store its K and V columns straight into
+// the fp16 cache slot `pos` of each of the m sequences instead of its output
+// (a 4-bit cache is appended by the decode attention, see AppendRow);
 // LnFuse makes the layer LayerNorm its finished rows [m][n] into `y` after a
 // grid-wide barrier (the launch is cooperative; `sync` = two ints of device
 // memory that are zero on entry and left zero).
 struct KvFuse {
-  uint8_t* k_codes;   // KvView layout of the m sequences' rows (bits == 16:
-  uint32_t* v_words;  // fp16 K / V rows, metas unused)
-  __half2* k_meta;
-  __half2* v_meta;
-  int h, heads, d, max_len, pos, bits;
+  __half* k;  // fp16 caches in the KvView layout of the m sequences
+  __half* v;
+  int h, heads, d, max_len, pos;
 };
 struct LnFuse {
   const __half* g;
@@ -125,6 +122,17 @@ size_t linear_workspace_bytes(int m, int n, int k, int w_bits, int force_splits)
 cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaStream_t s);
 
 // attention
+// The decode token's fp16 K and V rows ([b][ld], head j at columns j*d),
+// which the decode attention quantizes into cache slot `pos` before reading
+// the cache (4-bit caches; pos < 0: nothing to append).
+struct AppendRow {
+  const __half* k;
+  const __half* v;
+  int ld;
+  int pos;
+};
+constexpr AppendRow kNoAppend = {nullptr, nullptr, 0, -1};
+
 // Decode attention.  With part/ctr: when b * heads CTAs cannot fill the
 // GPU, each (sequence, head) is split over several CTAs
 // along the cache, partial results go to `part`
@@ -132,13 +140,13 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
 // ctr = b * heads ints, zero on entry and left zero.
 cudaError_t launch_attn_decode(const __half* q, int ldq, const KvView& kv, int b, int heads, int d,
                                int kv_bits, int len, __half* out, int ldo, float* part, int* ctr,
-                               cudaStream_t s);
+                               const AppendRow& app, cudaStream_t s);
 int attn_decode_splits(int b, int heads, int len);
 // Top-k sparse decode attention over a 4-bit cache: kk keys kept per
 // (sequence, head); idx (optional) receives the kept slots [b][heads][kk] in
 // ascending order.
 cudaError_t launch_attn_topk(const __half* q, int ldq, const KvView& kv, int b, int heads, int d, int len, int kk,
-                             __half* out, int ldo, int32_t* idx, cudaStream_t s);
+                             __half* out, int ldo, int32_t* idx, const AppendRow& app, cudaStream_t s);
 // ceil(len * permille / 1000), clamped to 1..len.
 inline int topk_count(int len, int permille) {
   const long long k = (static_cast<long long>(len) * permille + 999) / 1000;

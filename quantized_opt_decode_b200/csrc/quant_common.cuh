@@ -6,6 +6,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "kernels.h"
+
 namespace flexq {
 
 // Loads 32 consecutive fp16 values (64 B, 16-B aligned) as fp32; zeros when
@@ -73,6 +75,53 @@ __device__ __forceinline__ uint32_t pack_tiled(const uint32_t* q) {
 #pragma unroll
   for (int e = 0; e < 8; ++e) w |= (q[e] & 0xF) << (4 * ((e >> 1) + 4 * (e & 1)));
   return w;
+}
+
+// Quantize on append of one (sequence i, head j) at decode: the token's K and
+// V rows (d fp16 each) go to cache slot app.pos exactly as the append kernels
+// write them (K canonical codes, V the token's nibble in each
+// token-interleaved word, (min, scale) per 64 elements).  Called by one whole
+// warp; lanes 0 .. 2d/64 - 1 hold K (two per group), the next 2d/64 V.
+template <int D>
+__device__ __forceinline__ void append_row_q4(const AppendRow& app, const KvView& kv, int i, int j, int heads) {
+  constexpr int G = D / 64;
+  const int lane = threadIdx.x & 31;
+  const bool active = lane < 4 * G;
+  const bool is_v = lane >= 2 * G;
+  const int l2 = is_v ? lane - 2 * G : lane;
+  const int gd = l2 >> 1, half_id = l2 & 1;
+  const __half* src = (is_v ? app.v : app.k) + static_cast<size_t>(i) * app.ld + j * D + gd * 64 + half_id * 32;
+  float v[32];
+  load32(src, v, active);
+  uint32_t q[32];
+  __half m16, s16;
+  q64_lane_pair(v, q, m16, s16);
+  if (!active) return;
+  const size_t hr = static_cast<size_t>(i) * heads + j;
+  const size_t slot = hr * kv.max_len + app.pos;
+  if (!is_v) {
+    const uint4 out = make_uint4(pack_canonical(q), pack_canonical(q + 8), pack_canonical(q + 16),
+                                 pack_canonical(q + 24));
+    *reinterpret_cast<uint4*>(static_cast<uint8_t*>(kv.k) + slot * (D / 2) + gd * 32 + half_id * 16) = out;
+  } else {
+    uint4* w4 = reinterpret_cast<uint4*>(static_cast<uint32_t*>(kv.v) +
+                                         (hr * (kv_pad_len(kv.max_len) / 8) + app.pos / 8) * D + gd * 64 +
+                                         half_id * 32);
+    const int sh = 4 * (app.pos & 7);
+    const uint32_t clear = ~(0xFu << sh);
+    uint4 cur[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cur[u] = w4[u];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cur[u].x = (cur[u].x & clear) | (q[4 * u] << sh);
+      cur[u].y = (cur[u].y & clear) | (q[4 * u + 1] << sh);
+      cur[u].z = (cur[u].z & clear) | (q[4 * u + 2] << sh);
+      cur[u].w = (cur[u].w & clear) | (q[4 * u + 3] << sh);
+      w4[u] = cur[u];
+    }
+  }
+  if (half_id == 0) static_cast<__half2*>(is_v ? kv.v_meta : kv.k_meta)[slot * G + gd] = __halves2half2(m16, s16);
 }
 
 }  // namespace flexq

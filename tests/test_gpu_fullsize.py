@@ -18,8 +18,9 @@ b are multiples of the token tile), so ragged tiles are covered by the
 small-shape tests; what covers the other sequences here is a property that
 holds at any size: the kernels treat sequences independently and identically,
 so running the batch with its sequences rotated must give the rotated outputs
-bit for bit (prefill rotated by one sequence, decode by 17 sequences, which
-moves every token to another 16-token chunk of the GEMM epilogue).
+(prefill rotated by one sequence, decode by 17 sequences, which moves every
+token to another 16-token chunk of the GEMM epilogue), equal up to the order
+in which split tiles sum their fp32 partials (a few fp16 ulps).
 
 The decode step reads a cache that both sides fill from the same seeded fp16
 K/V rows through the quantizer (bit-exact, as the KV-append tests show):
@@ -41,7 +42,7 @@ pytestmark = pytest.mark.gpu
 
 import synth  # noqa: E402
 from oracle import opt, q64  # noqa: E402
-from gpu_helpers import assert_close, fq, rel_fro, to_host  # noqa: E402
+from gpu_helpers import assert_close, fq, rel_fro, to_host, ulp16  # noqa: E402
 from quantized_opt_decode_b200.device_model import DeviceModel, workspace  # noqa: E402
 
 TOL = 2e-3
@@ -88,6 +89,20 @@ def _check_codes(got_codes, want_codes, what):
     assert diff.max() <= 1 and (diff == 0).mean() > 0.99, (what, (diff == 0).mean(), diff.max())
 
 
+def _check_rotation(rot, ref, what):
+    """Rotating the batch rotates the outputs.  Where a linear layer splits
+    a tile's K range across CTAs (stream-K), the split points depend on the
+    tile, so a row that moves to another tile may sum its fp32 partials in
+    another order: allow a few fp16 ulps, far below any misplaced or wrong
+    row."""
+    rot = rot.astype(np.float64)
+    ref = ref.astype(np.float64)
+    err = np.abs(rot - ref)
+    bound = 8 * ulp16(ref) + 1e-4 * float(np.sqrt(np.mean(ref ** 2)))
+    k = int(np.argmax(err - bound))
+    assert (err <= bound).all(), f"{what} under rotation: element {k} off by {err.flat[k]:.3e}"
+
+
 @pytest.mark.parametrize("name", ["opt-1.3b", "opt-6.7b", "opt-30b", "opt-30b-s1024", "opt-175b"])
 def test_layer_full_size_sampled(name):
     p = dict(synth.CONFIGS[name])
@@ -114,11 +129,11 @@ def test_layer_full_size_sampled(name):
     y_got = to_host(yd.view(gb, s, h)[seqs][:, pos])
     k_shape = (gb, a, s + 1, d // 2) if p["kv_bits"] == 4 else (gb, a, s + 1, d)
     k_pre = to_host(dm.kv[0].k).reshape(k_shape)[seqs, :, :s]
-    # rotation by one sequence: the rotated outputs, bit for bit
+    # rotation by one sequence: the rotated outputs (up to split-tile summation order)
     y_rot = torch.empty_like(xd)
     fq.flexq_layer_prefill(dm.cfg, L, torch.roll(xd, s, 0), y_rot, kv, gb, s, ws, ws_n)
     fq.flexq_device_status()
-    assert torch.equal(torch.roll(y_rot, -s, 0), yd), "prefill is not invariant under rotating the batch"
+    _check_rotation(to_host(torch.roll(y_rot, -s, 0)), to_host(yd), "prefill")
     del y_rot
     # the decode reads a cache filled from seeded rows on both sides
     kvd = torch.empty(gb * s, 2 * h, dtype=torch.float16, device="cuda")
@@ -134,7 +149,7 @@ def test_layer_full_size_sampled(name):
     t3 = torch.empty_like(td)
     fq.flexq_layer_decode(dm.cfg, L, torch.roll(td, ROLL_DECODE, 0), t3, kv, gb, s, ws, ws_n)
     fq.flexq_device_status()
-    assert torch.equal(torch.roll(t3, -ROLL_DECODE, 0), t2), "decode is not invariant under rotating the batch"
+    _check_rotation(to_host(torch.roll(t3, -ROLL_DECODE, 0)), to_host(t2), "decode")
     del dm, xd, yd, kvd, kv_rot, ws
     torch.cuda.empty_cache()
 

@@ -189,7 +189,8 @@ def test_attention_decode_topk(h, heads, length, permille):
     for those heads the kept slots must equal the oracle's exactly and the
     output must meet the parity bar; for a head with a near-tie at the
     threshold the kept set must still be a valid top-k (k slots, each scoring
-    at least the oracle's k-th score minus the margin)."""
+    at least the oracle's k-th score minus the margin; the margin is ten times
+    the kernel's score rounding, and most heads have a clear gap)."""
     cfg = _cfg(h, heads, 4)
     b, L = 3, length + 3
     d = h // heads
@@ -218,7 +219,9 @@ def test_attention_decode_topk(h, heads, length, permille):
     for i in range(b):
         for j in range(heads):
             s = np.sort(sc[i, j])[::-1]
-            margin = 1e-3 * np.abs(s).max() + 1e-6
+            # the kernel's scores differ from float64 by about 2e-5 * max|s|
+            # (15-bit fixed-point q); 10x that decides a clear gap
+            margin = 2e-4 * np.abs(s).max() + 1e-6
             gi = got_idx[i, j]
             assert np.all(np.diff(gi) > 0) and gi.min() >= 0 and gi.max() < length
             if kk == length or s[kk - 1] - s[kk] > margin:
@@ -228,5 +231,5 @@ def test_attention_decode_topk(h, heads, length, permille):
                 n_clear += 1
             else:
                 assert np.all(sc[i, j][gi] >= s[kk - 1] - margin), (i, j)
-    assert n_clear >= 0.9 * b * heads
+    assert n_clear >= 0.7 * b * heads
     assert_close(np.stack(clear_got), np.stack(clear_ref), TOL, what=f"top-k attention L={length}")
