@@ -193,14 +193,33 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0, b = 255;
-      for (; b > 0; --b) {
-        if (above + hist[b] >= need) break;
-        above += hist[b];
+    if (warp == 0) {
+      // the bucket b from the top with (keys above b) < need <= (keys above
+      // b) + hist[b]: lane l owns bins 8l .. 8l+7, a suffix sum over lanes
+      // finds the lane, which then walks its own bins downwards
+      int cnt[8], own = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        cnt[k] = hist[lane * 8 + k];
+        own += cnt[k];
       }
-      pick[0] = static_cast<uint32_t>(b);
-      pick[1] = static_cast<uint32_t>(above);
+      int incl = own;  // keys in bins of lanes lane .. 31
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += n;
+      }
+      const int above_lane = incl - own;
+      const unsigned hit = __ballot_sync(0xffffffffu, above_lane < need && need <= incl);
+      if (lane == 31 - __clz(hit)) {  // the highest lane that holds the bucket
+        int above = above_lane, b = lane * 8 + 7;
+        for (int k = 7; k > 0; --k, --b) {
+          if (above + cnt[k] >= need) break;
+          above += cnt[k];
+        }
+        pick[0] = static_cast<uint32_t>(b);
+        pick[1] = static_cast<uint32_t>(above);
+      }
     }
     __syncthreads();
     need -= static_cast<int>(pick[1]);
