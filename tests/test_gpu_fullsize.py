@@ -20,7 +20,7 @@ holds at any size: the kernels treat sequences independently and identically,
 so running the batch with its sequences rotated must give the rotated outputs
 (prefill rotated by one sequence, decode by 17 sequences, which moves every
 token to another 16-token chunk of the GEMM epilogue), equal up to the order
-in which split tiles sum their fp32 partials (a few fp16 ulps).
+in which split tiles sum their fp32 partials (8 ulps + 1e-3 of the rms).
 
 The decode step reads a cache that both sides fill from the same seeded fp16
 K/V rows through the quantizer (bit-exact, as the KV-append tests show):
@@ -93,12 +93,13 @@ def _check_rotation(rot, ref, what):
     """Rotating the batch rotates the outputs.  Where a linear layer splits
     a tile's K range across CTAs (stream-K), the split points depend on the
     tile, so a row that moves to another tile may sum its fp32 partials in
-    another order: allow a few fp16 ulps, far below any misplaced or wrong
-    row."""
+    another order, and the difference passes through LayerNorm, GELU and a
+    second split GEMM: allow 8 fp16 ulps plus 1e-3 of the rms, far below the
+    O(1) error of a misplaced or wrong row."""
     rot = rot.astype(np.float64)
     ref = ref.astype(np.float64)
     err = np.abs(rot - ref)
-    bound = 8 * ulp16(ref) + 1e-4 * float(np.sqrt(np.mean(ref ** 2)))
+    bound = 8 * ulp16(ref) + 1e-3 * float(np.sqrt(np.mean(ref ** 2)))
     k = int(np.argmax(err - bound))
     assert (err <= bound).all(), f"{what} under rotation: element {k} off by {err.flat[k]:.3e}"
 
