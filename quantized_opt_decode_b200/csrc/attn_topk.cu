@@ -148,36 +148,56 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
       ql_o[w] |= static_cast<uint32_t>(io & 0xFF) << (8 * n);
     }
   }
+  // kUnroll groups of tokens are loaded before any is used, so each lane keeps
+  // several loads in flight (the pass is bound by load latency otherwise)
   float mx = -INFINITY;
-  constexpr int kStride = kTkThreads / 4;
-  for (int base = warp * 8; base < len; base += kStride) {
-    const int t = base + (lane >> 2);
-    const bool valid = t < len;
-    float partial = 0.f;
-    if (valid) {
-      uint32_t cw[NW];
+  constexpr int kStride = kTkThreads / 4;  // tokens per block-wide step
+  constexpr int kUnroll = 4;
+  for (int base = warp * 8; base < len; base += kUnroll * kStride) {
+    uint32_t cw[kUnroll][NW];
+    __half2 msh[kUnroll];
 #pragma unroll
-      for (int w = 0; w < NW; ++w) cw[w] = kw[static_cast<size_t>(t) * (D / 8) + cq * NW + w];
-      int dh = 0;
-      uint32_t dl = 0u;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const uint32_t lo = cw[w] & 0x0F0F0F0Fu, hi = (cw[w] >> 4) & 0x0F0F0F0Fu;
-        dh = __dp4a(static_cast<int>(lo), qh_e[w], dh);
-        dh = __dp4a(static_cast<int>(hi), qh_o[w], dh);
-        dl = __dp4a(lo, ql_e[w], dl);
-        dl = __dp4a(hi, ql_o[w], dl);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = base + u * kStride + (lane >> 2);
+      if (t < len) {
+        const uint32_t* src = kw + static_cast<size_t>(t) * (D / 8) + cq * NW;
+        if constexpr (NW == 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src);
+          cw[u][0] = v.x; cw[u][1] = v.y; cw[u][2] = v.z; cw[u][3] = v.w;
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2*>(src);
+          cw[u][0] = v.x; cw[u][1] = v.y;
+        }
+        msh[u] = km[static_cast<size_t>(t) * G + g];
       }
-      const float dot = (static_cast<float>(dh) * 256.0f + static_cast<float>(dl)) * inv_qscale;
-      const float2 ms = __half22float2(km[static_cast<size_t>(t) * G + g]);
-      partial = ms.y * dot + ms.x * qsum;
     }
-    partial += __shfl_xor_sync(0xffffffffu, partial, 1);
-    partial += __shfl_xor_sync(0xffffffffu, partial, 2);
-    if (valid) {
-      const float s = partial * inv_sqrt_d;
-      if (cq == 0) sc[t] = s;
-      mx = fmaxf(mx, s);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int t = base + u * kStride + (lane >> 2);
+      const bool valid = t < len;
+      float partial = 0.f;
+      if (valid) {
+        int dh = 0;
+        uint32_t dl = 0u;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          const uint32_t lo = cw[u][w] & 0x0F0F0F0Fu, hi = (cw[u][w] >> 4) & 0x0F0F0F0Fu;
+          dh = __dp4a(static_cast<int>(lo), qh_e[w], dh);
+          dh = __dp4a(static_cast<int>(hi), qh_o[w], dh);
+          dl = __dp4a(lo, ql_e[w], dl);
+          dl = __dp4a(hi, ql_o[w], dl);
+        }
+        const float dot = (static_cast<float>(dh) * 256.0f + static_cast<float>(dl)) * inv_qscale;
+        const float2 ms = __half22float2(msh[u]);
+        partial = ms.y * dot + ms.x * qsum;
+      }
+      partial += __shfl_xor_sync(0xffffffffu, partial, 1);
+      partial += __shfl_xor_sync(0xffffffffu, partial, 2);
+      if (valid) {
+        const float s = partial * inv_sqrt_d;
+        if (cq == 0) sc[t] = s;
+        mx = fmaxf(mx, s);
+      }
     }
   }
   const float M = block_max(mx, red);  // its barriers also publish sc[]
