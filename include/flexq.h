@@ -275,12 +275,14 @@ flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* lay
 /* Decode of one layer for the token at position pos of b sequences: t_dev,
  * y_dev fp16 [b][h] (distinct).  Appends this token's K/V to slot pos, then
  * attends over slots 0..pos read back from the cache.  For b <= 256 the
- * append happens inside the Q/K/V projection (its epilogue quantizes the
- * K/V columns straight into the cache: the same codes flexq_kv_append gives
- * those fp16 rows), LN2 runs inside the output projection (a cooperative
- * launch whose CTAs normalise the finished rows after a grid-wide barrier),
- * and decode attention splits each head's cache over several CTAs when
- * b * heads CTAs would not fill the GPU. */
+ * append needs no launch of its own: a 4-bit cache is appended by the
+ * decode attention kernel (one warp of each (sequence, head) CTA quantizes
+ * the token's K/V rows, the same codes flexq_kv_append gives those fp16
+ * rows, before the CTA reads the cache), an fp16 cache by the Q/K/V
+ * projection's epilogue; LN2 runs inside the output projection (a
+ * cooperative launch whose CTAs normalise the finished rows after a
+ * grid-wide barrier); decode attention splits each head's cache over several
+ * CTAs when b * heads CTAs would not fill the GPU. */
 flexq_status flexq_layer_decode(const flexq_config* cfg, const flexq_layer* layer,
                                 const void* t_dev, void* y_dev, const flexq_kv* kv, int b,
                                 int pos, void* ws_dev, size_t ws_bytes, void* stream);
@@ -331,8 +333,8 @@ flexq_status flexq_generate_prefill(const flexq_model* model, const int32_t* pro
  * With gpu_batch <= 256 each column is fused as in flexq_layer_decode, and
  * further: the embedding kernel applies layer 0's LN1, and every layer's FC2
  * kernel LayerNorms its output with the next layer's LN1 (the last layer's
- * with the final LayerNorm), so a layer is five kernels (QKV + append,
- * attention, output projection + LN, FC1 + GELU, FC2 + LN).  The split-tile
+ * with the final LayerNorm), so a layer is five kernels (QKV, attention with
+ * the append, output projection + LN, FC1 + GELU, FC2 + LN).  The split-tile
  * counters in the workspace are zeroed once per call and every kernel leaves
  * them zero; a kernel that gives up a bounded wait (FLEXQ_ERR_TIMEOUT) may
  * leave them dirty, so results of the rest of that call are undefined. */
@@ -434,9 +436,10 @@ typedef enum {
  * one host thread at a time).  stop synchronises `stream` and writes, per
  * kind, the summed device milliseconds and the number of bracketed calls
  * (an unfused linear layer's call also holds the memset of its split-tile
- * counters; a fused decode kernel counts under the kind of the linear layer
- * or embedding it belongs to: the K/V append under QKV, LN2 under OUT_PROJ,
- * the next LN1 or the final LayerNorm under FC2, layer 0's LN1 under EMBED). */
+ * counters; a fused decode kernel counts under the kind of the kernel it
+ * runs in: a 4-bit decode append under ATTN_DECODE (an fp16 one under QKV),
+ * LN2 under OUT_PROJ, the next LN1 or the final LayerNorm under FC2, layer
+ * 0's LN1 under EMBED). */
 flexq_status flexq_profile_start(void);
 flexq_status flexq_profile_stop(void* stream, float* total_ms /* [FLEXQ_K_COUNT] */,
                                 int* calls /* [FLEXQ_K_COUNT] */);
