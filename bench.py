@@ -378,6 +378,15 @@ class OracleSample:
         # one decode token of one sequence needs all l layers
         return self.b_o / (seconds * self.p["layers"])
 
+    def prefill_step(self, s_p: int) -> float:
+        """Layer-0 prefill of one sequence's first s_p prompt tokens (causal, so
+        it is exactly the prefill of an s_p-token prompt)."""
+        x = synth.normal_f16(synth.config_seed(self.p), synth.TID_TEST_BASE + 3, s_p * self.p["h"], 1.0)
+        x = x.reshape(1, s_p, self.p["h"]).astype(np.float64)
+        t0 = time.perf_counter()
+        self.opt.layer_prefill(self.cfg, self.W, x)
+        return time.perf_counter() - t0
+
 
 def cpu_cores():
     try:
@@ -400,12 +409,16 @@ def cpu_baseline(p: dict, budget_s: float = 12.0):
     while time.perf_counter() < t_end or len(times) < 3:
         times.append(smp.step())
     t = statistics.median(times)
+    s_p = min(p["s"], 128)
+    t_pre = smp.prefill_step(s_p)
     return {"value": round(smp.tokens_per_s(t), 4), "unit": "tokens/s", "cores": cpu_cores(),
             "kind": "oracle",
+            "prefill_value": round(s_p / (t_pre * p["layers"]), 4),
             "sample": (f"oracle (numpy float64) decode of layer 0 for {smp.b_o} sequences at KV "
                        f"length {smp.L + 1}, {len(times)} repetitions, median {t * 1e3:.1f} ms, "
-                       f"extrapolated x{p['layers']} layers per token; setup {setup:.0f} s "
-                       "(weights drawn, quantized, dequantized on the host)")}
+                       f"extrapolated x{p['layers']} layers per token; prefill_value: layer-0 "
+                       f"prefill of one {s_p}-token prompt, {t_pre:.2f} s, extrapolated the same "
+                       f"way; setup {setup:.0f} s (weights drawn, quantized, dequantized on the host)")}
 
 
 def run_reference(args, p):
@@ -658,7 +671,7 @@ def run_offload(args, p):
     torch.cuda.empty_cache()
     peaks = load_peaks()
     free, _ = torch.cuda.mem_get_info()
-    hw = fq.flexq_hw(h2d_gbps=h2d, hbm_gbps=peaks["hbm_gbps"], tensor_tflops=peaks["bf16_tflops_sustained"],
+    hw = fq.flexq_hw(h2d_gbps=h2d, hbm_gbps=peaks["hbm_gbs"], tensor_tflops=peaks["bf16_tflops_sustained"],
                      device_bytes=free - 6e9)
     ch = fq.flexq_offload_plan(dm.struct, s, n, hw, args.max_block)
     gbs, b = ch.gpu_batch, ch.gpu_batch * ch.num_batches
