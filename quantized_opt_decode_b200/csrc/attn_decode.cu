@@ -118,12 +118,6 @@ __global__ void __launch_bounds__(kThreads, 8) attn_decode_q4_kernel(const __hal
   const __half2* vm = static_cast<const __half2*>(kv.v_meta) + hr * kv.max_len * G;
   const uint32_t* vw = static_cast<const uint32_t*>(kv.v) + hr * (kv_pad_len(kv.max_len) / 8) * D;
 
-  // decode: this token's K/V rows enter the cache before the passes read it
-  if (app.pos >= 0) {
-    if (warp == 0) append_row_q4<D>(app, kv, i, j, heads);
-    __syncthreads();
-  }
-
   // q slice of this lane as fp32, its sum, and the fixed-point bytes
   float qf[DPL];
   const __half* qp = q + static_cast<size_t>(i) * ldq + j * D + c * DPL;
@@ -132,6 +126,12 @@ __global__ void __launch_bounds__(kThreads, 8) attn_decode_q4_kernel(const __hal
     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(qp + e));
     qf[e] = f.x;
     qf[e + 1] = f.y;
+  }
+
+  // decode: this token's K/V rows enter the cache before the passes read it
+  if (app.pos >= 0) {
+    append_group_q4<D>(app, kv, i, j, heads, warp, lane);
+    __syncthreads();
   }
   float qsum = 0.f, qmax = 0.f;
 #pragma unroll

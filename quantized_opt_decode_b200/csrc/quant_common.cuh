@@ -80,48 +80,57 @@ __device__ __forceinline__ uint32_t pack_tiled(const uint32_t* q) {
 // Quantize on append of one (sequence i, head j) at decode: the token's K and
 // V rows (d fp16 each) go to cache slot app.pos exactly as the append kernels
 // write them (K canonical codes, V the token's nibble in each
-// token-interleaved word, (min, scale) per 64 elements).  Called by one whole
-// warp; lanes 0 .. 2d/64 - 1 hold K (two per group), the next 2d/64 V.
+// token-interleaved word, (min, scale) per 64 elements).  One warp per
+// 64-element group: warp w < d/64 takes K group w, the next d/64 warps the V
+// groups, two elements per lane (the group's min and max by warp shuffles,
+// which give the same values as any other order); warps past 2d/64 return.
+// A V warp fetches the token's interleaved words together with its fp16 pair,
+// so the two reads overlap.  The caller synchronises before reading the slot.
 template <int D>
-__device__ __forceinline__ void append_row_q4(const AppendRow& app, const KvView& kv, int i, int j, int heads) {
+__device__ __forceinline__ void append_group_q4(const AppendRow& app, const KvView& kv, int i, int j, int heads,
+                                                int warp, int lane) {
   constexpr int G = D / 64;
-  const int lane = threadIdx.x & 31;
-  const bool active = lane < 4 * G;
-  const bool is_v = lane >= 2 * G;
-  const int l2 = is_v ? lane - 2 * G : lane;
-  const int gd = l2 >> 1, half_id = l2 & 1;
-  const __half* src = (is_v ? app.v : app.k) + static_cast<size_t>(i) * app.ld + j * D + gd * 64 + half_id * 32;
-  float v[32];
-  load32(src, v, active);
-  uint32_t q[32];
-  __half m16, s16;
-  q64_lane_pair(v, q, m16, s16);
-  if (!active) return;
+  if (warp >= 2 * G) return;
+  const bool is_v = warp >= G;
+  const int gd = is_v ? warp - G : warp;
   const size_t hr = static_cast<size_t>(i) * heads + j;
   const size_t slot = hr * kv.max_len + app.pos;
+  uint2* vp = nullptr;
+  uint2 vold = make_uint2(0u, 0u);
+  if (is_v) {
+    vp = reinterpret_cast<uint2*>(static_cast<uint32_t*>(kv.v) +
+                                  (hr * (kv_pad_len(kv.max_len) / 8) + app.pos / 8) * D + gd * 64 + 2 * lane);
+    vold = *vp;
+  }
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(
+      (is_v ? app.v : app.k) + static_cast<size_t>(i) * app.ld + j * D + gd * 64 + 2 * lane));
+  float lo = fminf(f.x, f.y), hi = fmaxf(f.x, f.y);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  lo = __fadd_rn(lo, 0.0f);  // -0 -> +0
+  hi = __fadd_rn(hi, 0.0f);
+  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
+  const __half m16 = __float2half_rn(lo);
+  const float sc = __half2float(s16);
+  const float mn = __half2float(m16);
+  uint32_t c0 = 0u, c1 = 0u;
+  if (sc != 0.0f) {
+    c0 = static_cast<uint32_t>(fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(f.x, mn), sc)), 0.0f), 15.0f));
+    c1 = static_cast<uint32_t>(fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(f.y, mn), sc)), 0.0f), 15.0f));
+  }
   if (!is_v) {
-    const uint4 out = make_uint4(pack_canonical(q), pack_canonical(q + 8), pack_canonical(q + 16),
-                                 pack_canonical(q + 24));
-    *reinterpret_cast<uint4*>(static_cast<uint8_t*>(kv.k) + slot * (D / 2) + gd * 32 + half_id * 16) = out;
+    static_cast<uint8_t*>(kv.k)[slot * (D / 2) + gd * 32 + lane] = static_cast<uint8_t>(c0 | (c1 << 4));
   } else {
-    uint4* w4 = reinterpret_cast<uint4*>(static_cast<uint32_t*>(kv.v) +
-                                         (hr * (kv_pad_len(kv.max_len) / 8) + app.pos / 8) * D + gd * 64 +
-                                         half_id * 32);
     const int sh = 4 * (app.pos & 7);
     const uint32_t clear = ~(0xFu << sh);
-    uint4 cur[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) cur[u] = w4[u];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      cur[u].x = (cur[u].x & clear) | (q[4 * u] << sh);
-      cur[u].y = (cur[u].y & clear) | (q[4 * u + 1] << sh);
-      cur[u].z = (cur[u].z & clear) | (q[4 * u + 2] << sh);
-      cur[u].w = (cur[u].w & clear) | (q[4 * u + 3] << sh);
-      w4[u] = cur[u];
-    }
+    vold.x = (vold.x & clear) | (c0 << sh);
+    vold.y = (vold.y & clear) | (c1 << sh);
+    *vp = vold;
   }
-  if (half_id == 0) static_cast<__half2*>(is_v ? kv.v_meta : kv.k_meta)[slot * G + gd] = __halves2half2(m16, s16);
+  if (lane == 0) static_cast<__half2*>(is_v ? kv.v_meta : kv.k_meta)[slot * G + gd] = __halves2half2(m16, s16);
 }
 
 }  // namespace flexq
