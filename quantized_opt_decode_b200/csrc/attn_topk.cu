@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
   constexpr int NW = DPL / 8;
   constexpr int DPV = D / 32;
   extern __shared__ float sc[];                                  // [len] scores
-  uint8_t* sel = reinterpret_cast<uint8_t*>(sc + ((len + 3) & ~3));  // [len] kept flags
+  int* blist = reinterpret_cast<int*>(sc + ((len + 3) & ~3));     // [nblk] blocks holding a kept key
+  uint8_t* sel = reinterpret_cast<uint8_t*>(blist + (((len + 7) / 8 + 3) & ~3));  // [len] kept flags
   __shared__ int hist[256];
   __shared__ int scan[kTkWarps];
   __shared__ float red[kTkWarps];
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
 
   // decode: this token's K/V rows enter the cache before the scores read it
   if (app.pos >= 0) {
-    if (warp == 0) append_row_q4<D>(app, kv, i, j, heads);
+    append_group_q4<D>(app, kv, i, j, heads, warp, lane);
     __syncthreads();
   }
 
@@ -208,9 +209,16 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = threadIdx.x; b < 256; b += kTkThreads) hist[b] = 0;
     __syncthreads();
-    for (int t = threadIdx.x; t < len; t += kTkThreads) {
-      const uint32_t key = order_key(sc[t]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    // lanes that hit the same bin add once, by their lowest lane (the
+    // scores cluster in a few bins per pass, so plain atomics would serialise)
+    for (int t0 = 0; t0 < len; t0 += kTkThreads) {
+      const int t = t0 + threadIdx.x;
+      uint32_t key = 0u;
+      if (t < len) key = order_key(sc[t]);
+      const bool act = t < len && (key & mask) == prefix;
+      const int bin = act ? static_cast<int>((key >> shift) & 255u) : 256 + lane;
+      const unsigned same = __match_any_sync(0xffffffffu, bin);
+      if (act && __ffs(same) - 1 == lane) atomicAdd(&hist[bin], __popc(same));
     }
     __syncthreads();
     if (warp == 0) {
@@ -304,47 +312,75 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
       if (sel[t]) dst[at++] = t;
   }
 
-  // ---- values of the blocks holding a kept token
+  // ---- the 8-token blocks holding a kept token, in ascending order
+  const int nblk = (len + 7) / 8;
+  int n_kb = 0;
+  for (int b0 = 0; b0 < nblk; b0 += kTkThreads) {
+    const int blk = b0 + threadIdx.x;
+    int any = 0;
+    if (blk < nblk)
+      for (int k = 0; k < 8 && blk * 8 + k < len; ++k) any |= sel[blk * 8 + k];
+    int cnt = 0;
+    const int at = block_exclusive_scan(any, scan, &cnt);
+    if (any) blist[n_kb + at] = blk;
+    n_kb += cnt;
+  }
+  __syncthreads();
+
+  // ---- values of those blocks; kVU blocks' words in flight per lane
+  constexpr int kVU = 4;
   const int gv = (lane * DPV) / 64;
   uint32_t al[DPV], ah[DPV];
 #pragma unroll
   for (int e = 0; e < DPV; ++e) al[e] = ah[e] = 0u;
-  const int nblk = (len + 7) / 8;
-  for (int blk = warp; blk < nblk; blk += kTkWarps) {
-    // lane k < 8 * G: token 8 blk + (k & 7), group k >> 3
-    const int tk = blk * 8 + (lane & 7);
-    const int gk = lane >> 3;
-    const bool kept = lane < 8 * G && tk < len && sel[tk];
-    if (__ballot_sync(0xffffffffu, kept) == 0u) continue;
-    uint32_t wi = 0u;
-    if (kept) {
-      const float p = __expf(sc[tk] - M);
-      const float sv = __high2float(vm[static_cast<size_t>(tk) * G + gk]);
-      const float wqk = stat[G + gk] > 0.f ? 65535.0f / stat[G + gk] : 0.f;
-      wi = min(65535u, __float2uint_rn(p * sv * wqk));
-    }
-    uint32_t le = 0u, lo = 0u, he = 0u, ho = 0u;
+  for (int r0 = warp; r0 < n_kb; r0 += kVU * kTkWarps) {
+    uint32_t words[kVU][DPV];
+    int blks[kVU];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t w = __shfl_sync(0xffffffffu, wi, gv * 8 + k);
-      const int sh = 8 * (k >> 1);
-      if (k & 1) {
-        lo |= (w & 0xFFu) << sh;
-        ho |= (w >> 8) << sh;
-      } else {
-        le |= (w & 0xFFu) << sh;
-        he |= (w >> 8) << sh;
+    for (int u = 0; u < kVU; ++u) {
+      const int r = r0 + u * kTkWarps;
+      blks[u] = r < n_kb ? blist[r] : -1;
+      if (blks[u] >= 0) {
+        const uint32_t* src = vw + static_cast<size_t>(blks[u]) * D + lane * DPV;
+#pragma unroll
+        for (int e = 0; e < DPV; ++e) words[u][e] = src[e];
       }
     }
-    const uint32_t* src = vw + static_cast<size_t>(blk) * D + lane * DPV;
 #pragma unroll
-    for (int e = 0; e < DPV; ++e) {
-      const uint32_t word = src[e];
-      const uint32_t lo4 = word & 0x0F0F0F0Fu, hi4 = (word >> 4) & 0x0F0F0F0Fu;
-      al[e] = __dp4a(lo4, le, al[e]);
-      al[e] = __dp4a(hi4, lo, al[e]);
-      ah[e] = __dp4a(lo4, he, ah[e]);
-      ah[e] = __dp4a(hi4, ho, ah[e]);
+    for (int u = 0; u < kVU; ++u) {
+      if (blks[u] < 0) break;  // warp-uniform
+      // lane k < 8 * G: token 8 blk + (k & 7), group k >> 3
+      const int tk = blks[u] * 8 + (lane & 7);
+      const int gk = lane >> 3;
+      const bool kept = lane < 8 * G && tk < len && sel[tk];
+      uint32_t wi = 0u;
+      if (kept) {
+        const float p = __expf(sc[tk] - M);
+        const float sv = __high2float(vm[static_cast<size_t>(tk) * G + gk]);
+        const float wqk = stat[G + gk] > 0.f ? 65535.0f / stat[G + gk] : 0.f;
+        wi = min(65535u, __float2uint_rn(p * sv * wqk));
+      }
+      uint32_t le = 0u, lo = 0u, he = 0u, ho = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t w = __shfl_sync(0xffffffffu, wi, gv * 8 + k);
+        const int sh = 8 * (k >> 1);
+        if (k & 1) {
+          lo |= (w & 0xFFu) << sh;
+          ho |= (w >> 8) << sh;
+        } else {
+          le |= (w & 0xFFu) << sh;
+          he |= (w >> 8) << sh;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < DPV; ++e) {
+        const uint32_t lo4 = words[u][e] & 0x0F0F0F0Fu, hi4 = (words[u][e] >> 4) & 0x0F0F0F0Fu;
+        al[e] = __dp4a(lo4, le, al[e]);
+        al[e] = __dp4a(hi4, lo, al[e]);
+        ah[e] = __dp4a(lo4, he, ah[e]);
+        ah[e] = __dp4a(hi4, ho, ah[e]);
+      }
     }
   }
 #pragma unroll
@@ -364,7 +400,8 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
 template <int D>
 cudaError_t launch_topk(const __half* q, int ldq, const KvView& kv, int b, int heads, int len, int kk, __half* out,
                         int ldo, int32_t* idx, const AppendRow& app, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>((len + 3) & ~3) * sizeof(float) + static_cast<size_t>((len + 15) & ~15);
+  const size_t smem = static_cast<size_t>((len + 3) & ~3) * sizeof(float) +
+                      static_cast<size_t>(((len + 7) / 8 + 3) & ~3) * sizeof(int) + static_cast<size_t>((len + 15) & ~15);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(attn_topk_q4_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
