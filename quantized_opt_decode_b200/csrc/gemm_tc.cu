@@ -11,22 +11,27 @@
 //
 // One output tile = 128 features x up to 256 tokens; the weight is the MMA's A
 // operand, so a small decode batch becomes the MMA's N.  A persistent CTA per
-// SM walks a list of (tile, k-block range) segments:
-//   warp 0      TMA producer: per pipeline stage one cp.async.bulk of the
-//               packed weight chunks (codes + min/scale, 4608 contiguous bytes
-//               per 64-wide k-block) and one 128-byte-swizzled
-//               cp.async.bulk.tensor box of the activations per k-block;
-//   warps 2-9   dequantize the weight rows into a shared-memory ring of fp16
-//               A tiles in the UMMA K-major SW128 layout ((code | 0x6400) is
-//               the fp16 value 1024 + code; one half2 subtract and one half2
-//               fused multiply-add give code * scale + min rounded once);
+// SM walks a list of (tile, k-block range) segments in k-steps of KS 64-wide
+// k-blocks:
+//   warp 0      weight producer: per k-step one cp.async.bulk of the KS packed
+//               chunks (codes + min/scale, 4608 contiguous bytes per k-block),
+//               or one 3-D tensor box of fp16 weights;
+//   warp 14     activation producer: per k-step one 3-D tensor box {64 columns,
+//               tokens, KS k-blocks}, i.e. KS 128-byte-swizzled tiles;
+//   warps 2-9   dequantize the weight rows ((code | 0x6400) is the fp16 value
+//               1024 + code; one half2 subtract and one half2 fused multiply-
+//               add give code * scale + min rounded once): decode-sized tiles
+//               into tensor memory (tcgen05.st, one weight row per TMEM lane),
+//               larger tiles into a shared-memory ring in the UMMA K-major
+//               SW128 layout;
 //   warp 1      owns TMEM and, from one thread, issues tcgen05.mma.kind::f16
-//               (M=128, N=tokens, K=16; A and B from shared memory);
+//               (M=128, N=tokens, K=16; A from tensor or shared memory, B from
+//               shared memory);
 //   warps 10-13 epilogue (below).
-// Decode-sized tiles (<= 160 tokens) on 4-bit weights move two k-blocks per
-// stage when K allows (half the mbarrier hand-offs per FLOP); fp16 weights
-// (the LM head, fp16-weight configurations) arrive by TMA and skip the
-// dequantizing warps.
+// A copying thread completes about one copy per memory round trip whatever
+// its size (up to ~16 KB), so each ring has its own thread and every copy
+// moves a whole k-step: KS = 4 for 4-bit decode tiles of <= 128 tokens, 2 for
+// other decode tiles, 1 for prefill tiles.
 //
 // Epilogue (warps 10-13, one TMEM lane quarter each): tcgen05.ld, + bias,
 // GELU, + residual, fp16 or fp32 store; two accumulator buffers let it overlap
@@ -50,10 +55,11 @@
 namespace flexq {
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;  // 15 warps: W producer, MMA, 8 dequantizing, 4 epilogue, B producer
 constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
+constexpr int kBWarp = 14;
 constexpr int kATileBytes = 128 * 64 * 2;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
@@ -85,6 +91,7 @@ struct GemmParams {
   uint32_t w_slot_bytes, b_slot_bytes;
   uint32_t acc_cols;    // TMEM columns between the two accumulator buffers
   uint32_t tmem_alloc;  // columns allocated (power of two)
+  uint32_t a_col0;      // first TMEM column of the dequantized A ring (A in tensor memory)
   Sched sc;
   const __half* bias;
   const __half* residual;
@@ -657,28 +664,33 @@ struct StepCursor {
 };
 
 // KS: 64-wide k-blocks per k-step (two halve the mbarrier hand-offs per
-// tile, which bound decode-sized tiles).  Three rings in shared memory:
-//   W  weight chunks (4-bit: the packed codes + (min, scale); fp16: TMA tiles
-//      that are the MMA's A operand directly), filled by the producer far
-//      ahead of use: the weights stream from HBM, so the bytes this SM keeps
-//      in flight set the rate at which it receives them;
-//   B  activation boxes (from L2, a short ring);
-//   A  dequantized fp16 tiles (4-bit only), written by the dequantizing warps.
-// The producer issues in the order W(0 .. SW-1), then B(i), W(i + SW) for
-// i = 0, 1, ..: B(i) waits for the MMA of step i - SB, W(i + SW) for the
-// dequantizing warps to have read step i (they release a W slot as soon as
-// its codes are in registers), so the weight ring runs a whole ring ahead.
-template <bool kW4, int KS>
+// tile, which bound decode-sized tiles).  Three rings:
+//   W  weight chunks in shared memory (4-bit: the packed codes + (min,
+//      scale); fp16: TMA tiles that are the MMA's A operand directly), filled
+//      by the producer far ahead of use: the weights stream from HBM, so the
+//      bytes this SM keeps in flight set the rate at which it receives them;
+//   B  activation boxes in shared memory (from L2, a short ring);
+//   A  dequantized fp16 tiles (4-bit only), written by the dequantizing warps:
+//      in shared memory, or with kTA in tensor memory (tcgen05.st, one weight
+//      row per TMEM lane), read there by the MMA.  Decode-sized tiles use
+//      kTA: the shared-memory port then carries only the copies, the code
+//      reads and the MMA's B reads, not 2 x 16 KB of A per k-block.
+// Each ring has its own issuing thread: B(i) waits for the MMA of step
+// i - SB, W(i) for the dequantizing warps to have read step i - SW (they
+// release a W slot as soon as its codes are in registers; with fp16 weights
+// the MMA releases it), so the weight ring runs a whole ring ahead.
+template <bool kW4, int KS, bool kTA>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                    const GemmParams p) {
+  static_assert(!kTA || (kW4 && (KS == 2 || KS == 4)), "A in tensor memory: 4-bit weights, 2 or 4 k-blocks per step");
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int SW = p.w_stages, SB = p.b_stages, SA = p.a_stages;
   constexpr uint32_t a_slot_bytes = KS * kATileBytes;
-  uint8_t* a_ring = smem;                                // SA x KS fp16 A tiles (4-bit weights only)
-  uint8_t* w_ring = a_ring + SA * a_slot_bytes;          // SW x w_slot_bytes
+  uint8_t* a_ring = smem;                                         // SA x KS fp16 A tiles (4-bit, !kTA)
+  uint8_t* w_ring = a_ring + (kTA ? 0 : SA * a_slot_bytes);       // SW x w_slot_bytes
   uint8_t* b_ring = w_ring + SW * p.w_slot_bytes;        // SB x b_slot_bytes
   uint8_t* region = b_ring + SB * p.b_slot_bytes;
   uint64_t* wfull = reinterpret_cast<uint64_t*>(region);
@@ -726,76 +738,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *c.tmem_slot;
   const Sched& sc = p.sc;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == kBWarp) {
+    // ------------------------------------------------------------ producers
+    // Two issuing threads, one per ring: a thread completes about one copy
+    // per HBM/L2 round trip whatever its size (up to ~16 KB), so the weight
+    // stream and the activation stream each get their own, and every copy
+    // moves a whole k-step (KS k-blocks: one bulk copy of the packed chunks,
+    // one 3-D tensor box of the activations or fp16 weights).
     if (lane == 0) {
-      prefetch_tmap(&tmap_x);
-      if (!kW4) prefetch_tmap(&tmap_w);
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
-      const uint32_t w_tx = KS * (kW4 ? static_cast<uint32_t>(kTileBytes) : static_cast<uint32_t>(kATileBytes));
-      const uint32_t b_tx = KS * b_bytes;
-      StepCursor wc, bc;
-      wc.start(sc, cta);
-      bc.start(sc, cta);
-      Ring rw, rb;
-      int nw = 0, nb = 0;
-      bool stop = false;
-      auto slot_free = [&](uint64_t* bar, const Ring& r) {
-        if (!mbar_wait(bar, r.ph ^ 1u, p.wait_ns)) {
+      const bool w_role = warp == 0;
+      const uint64_t pol = w_role ? policy_evict_first() : policy_evict_last();
+      if (w_role && !kW4) prefetch_tmap(&tmap_w);
+      if (!w_role) prefetch_tmap(&tmap_x);
+      const int S = w_role ? SW : SB;
+      uint64_t* full = w_role ? wfull : bfull;
+      uint64_t* empty = w_role ? wempty : bempty;
+      uint8_t* ring = w_role ? w_ring : b_ring;
+      const uint32_t slot_bytes = w_role ? p.w_slot_bytes : p.b_slot_bytes;
+      const uint32_t tx = w_role ? KS * (kW4 ? static_cast<uint32_t>(kTileBytes) : static_cast<uint32_t>(kATileBytes))
+                                 : KS * b_bytes;
+      StepCursor cur;
+      cur.start(sc, cta);
+      Ring r;
+      int n = 0;
+      while (cur.valid) {
+        if (!mbar_wait(&empty[r.s], r.ph ^ 1u, p.wait_ns)) {
           set_error(p.err, DEV_TIMEOUT_PRODUCER);
           *c.abort_flag = 1;
         }
-        return *c.abort_flag == 0;
-      };
-      auto issue_w = [&]() {
-        if (!slot_free(&wempty[rw.s], rw)) return false;
-        const int n_tile = wc.g.tile % sc.n_tiles;
-        uint8_t* dst = w_ring + rw.s * p.w_slot_bytes;
-        mbar_arrive_expect_tx(&wfull[rw.s], w_tx);
-        if (kW4) {
-          bulk_load(dst, p.wq + (static_cast<size_t>(n_tile) * p.kb_real + wc.ks * KS) * kTileBytes, KS * kTileBytes,
-                    &wfull[rw.s], pol_w);
+        if (*c.abort_flag) break;
+        uint8_t* dst = ring + r.s * slot_bytes;
+        mbar_arrive_expect_tx(&full[r.s], tx);
+        if (!w_role) {
+          tma_load_3d(dst, &tmap_x, &full[r.s], 0, (cur.g.tile / sc.n_tiles) * p.tok_tile, cur.ks * KS, pol);
+        } else if (kW4) {
+          const int n_tile = cur.g.tile % sc.n_tiles;
+          bulk_load(dst, p.wq + (static_cast<size_t>(n_tile) * p.kb_real + cur.ks * KS) * kTileBytes, KS * kTileBytes,
+                    &full[r.s], pol);
         } else {
-#pragma unroll
-          for (int u = 0; u < KS; ++u)
-            tma_load_2d(dst + u * kATileBytes, &tmap_w, &wfull[rw.s], (wc.ks * KS + u) * 64, n_tile * 128, pol_w);
+          tma_load_3d(dst, &tmap_w, &full[r.s], 0, (cur.g.tile % sc.n_tiles) * 128, cur.ks * KS, pol);
         }
-        rw.next(SW);
-        ++nw;
-        wc.next(sc, cta);
-        return true;
-      };
-      auto issue_b = [&]() {
-        if (!slot_free(&bempty[rb.s], rb)) return false;
-        const int t_row = (bc.g.tile / sc.n_tiles) * p.tok_tile;
-        uint8_t* dst = b_ring + rb.s * p.b_slot_bytes;
-        mbar_arrive_expect_tx(&bfull[rb.s], b_tx);
-#pragma unroll
-        for (int u = 0; u < KS; ++u)
-          tma_load_2d(dst + u * b_bytes, &tmap_x, &bfull[rb.s], (bc.ks * KS + u) * 64, t_row, pol_x);
-        rb.next(SB);
-        ++nb;
-        bc.next(sc, cta);
-        return true;
-      };
-      while (!stop && wc.valid && nw < SW) stop = !issue_w();
-      while (!stop && bc.valid) {
-        stop = !issue_b();
-        if (!stop && wc.valid) stop = !issue_w();
+        r.next(S);
+        ++n;
+        cur.next(sc, cta);
       }
       // Never leave the CTA with bulk copies still landing in its shared memory.
-      for (int j = max(0, nw - SW); j < nw; ++j)
-        mbar_wait(&wfull[j % SW], static_cast<uint32_t>(j / SW) & 1u, drain_ns(p.wait_ns));
-      for (int j = max(0, nb - SB); j < nb; ++j)
-        mbar_wait(&bfull[j % SB], static_cast<uint32_t>(j / SB) & 1u, drain_ns(p.wait_ns));
+      for (int j = max(0, n - S); j < n; ++j)
+        mbar_wait(&full[j % S], static_cast<uint32_t>(j / S) & 1u, drain_ns(p.wait_ns));
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
       // descriptors of slot 0; a slot is reached by adding its byte offset >> 4
-      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(kW4 ? a_ring : w_ring));
+      const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(kW4 && !kTA ? a_ring : w_ring));
+      const uint32_t a_tmem0 = tmem_base + p.a_col0;
       const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(b_ring));
       const uint32_t a_step = (kW4 ? a_slot_bytes : p.w_slot_bytes) >> 4;
       const uint32_t b_step = p.b_slot_bytes >> 4;
@@ -825,14 +822,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             stop = true;
             break;
           }
-          const uint64_t adesc = adesc0 + static_cast<uint64_t>(ra.s * a_step);
           const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(rb.s * b_step);
+          if constexpr (kTA) {
+            tc_fence_after();  // the dequantizing warps' tensor-memory stores
+            const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(ra.s * KS * 32);
 #pragma unroll
-          for (int u = 0; u < KS; ++u)
+            for (int u = 0; u < KS; ++u)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_f16_ss(d_tmem, adesc + u * (kATileBytes >> 4) + 2 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk, idesc,
-                         (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                mma_f16_ts(d_tmem, a_tmem + u * 32 + 8 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk, idesc,
+                           (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            const uint64_t adesc = adesc0 + static_cast<uint64_t>(ra.s * a_step);
+#pragma unroll
+            for (int u = 0; u < KS; ++u)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_f16_ss(d_tmem, adesc + u * (kATileBytes >> 4) + 2 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk,
+                           idesc, (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(&bempty[rb.s]);
           mma_commit(kW4 ? &aempty[ra.s] : &wempty[ra.s]);
         }
@@ -846,7 +854,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------------------ dequantize
-    if (kW4) {
+    if constexpr (kTA) {
+      // warp w stores TMEM lanes 32 (w % 4) ..: one weight row per thread;
+      // the two warps of a lane quarter take alternate k-blocks of the step
+      constexpr int KU = KS / 2;  // k-blocks per thread and step
+      const int quarter = warp & 3;
+      const int grp = (warp - 2) >> 2;
+      const int row = quarter * 32 + lane;
+      const uint32_t t_row = tmem_base + p.a_col0 + (static_cast<uint32_t>(quarter * 32) << 16);
+      Ring rw, ra;
+      Seg g;
+      bool stop = false;
+      for (int q = 0; !stop && get_seg(sc, cta, q, g); ++q) {
+        for (int ks = g.kb0; ks < g.kb1; ++ks, rw.next(SW), ra.next(SA)) {
+          bool ok = mbar_wait(&wfull[rw.s], rw.ph, p.wait_ns);
+          ok = ok && mbar_wait(&aempty[ra.s], ra.ph ^ 1u, p.wait_ns);
+          if (!ok) {
+            set_error(p.err, DEV_TIMEOUT_CONSUMER);
+            *c.abort_flag = 1;
+          }
+          // warp-uniform: the tensor-memory store below is a warp-wide instruction
+          if (__any_sync(0xffffffffu, !ok || *c.abort_flag)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();  // the MMAs that read this A slot have completed
+          uint4 c0[KU], c1[KU];
+          __half2 mm[KU];
+#pragma unroll
+          for (int v = 0; v < KU; ++v) {
+            const uint8_t* raw = w_ring + rw.s * p.w_slot_bytes + (grp + 2 * v) * kTileBytes;
+            c0[v] = *reinterpret_cast<const uint4*>(raw + row * 32);
+            c1[v] = *reinterpret_cast<const uint4*>(raw + row * 32 + 16);
+            mm[v] = *reinterpret_cast<const __half2*>(raw + kTileCodeBytes + row * 4);
+          }
+          // the codes are in registers: the weight slot may be refilled
+          mbar_arrive(&wempty[rw.s]);
+#pragma unroll
+          for (int v = 0; v < KU; ++v) {
+            const __half2 m2 = __low2half2(mm[v]);
+            const __half2 s2 = __high2half2(mm[v]);
+            const uint32_t words[8] = {c0[v].x, c0[v].y, c0[v].z, c0[v].w, c1[v].x, c1[v].y, c1[v].z, c1[v].w};
+            uint32_t r[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint4 d = dequant8(words[j], s2, m2);
+              r[4 * j] = d.x;
+              r[4 * j + 1] = d.y;
+              r[4 * j + 2] = d.z;
+              r[4 * j + 3] = d.w;
+            }
+            __syncwarp();
+            tmem_st_x32(t_row + static_cast<uint32_t>(ra.s * KS * 32 + (grp + 2 * v) * 32), r);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&afull[ra.s]);
+        }
+      }
+    } else if (kW4) {
       const int ct = threadIdx.x - 64;
       const int row = ct >> 1;
       const int hf = ct & 1;
@@ -892,7 +958,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
+  } else if (warp < kEpiWarp0 + 4) {
     epilogue_role(p, c, tmem_base, warp, lane);
   }
   teardown(p, c, tmem_base, warp);
@@ -920,16 +986,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D fp16 tensor [rows][cols] with row stride ld (elements), box 64 x box_rows,
-// 128-byte swizzle, zero fill out of bounds.
-bool encode_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
+// fp16 matrix [rows][cols] (row stride ld elements, cols a multiple of 64)
+// viewed as [cols / 64][rows][64]: a box {64, box_rows, box_kb} is box_kb
+// consecutive 64-column blocks, each a 128-byte-swizzled [box_rows][64] tile
+// (the UMMA K-major layout), stacked in shared memory; zero fill out of bounds.
+bool encode_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows, int box_kb) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(cols / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_kb)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -939,9 +1007,10 @@ bool encode_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld,
 // the address, extents, stride and box, so a key always yields the same map.
 struct TmapKey {
   const void* base;
-  int rows, cols, ld, box_rows;
+  int rows, cols, ld, box_rows, box_kb;
   bool operator==(const TmapKey& o) const {
-    return base == o.base && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows;
+    return base == o.base && rows == o.rows && cols == o.cols && ld == o.ld && box_rows == o.box_rows &&
+           box_kb == o.box_kb;
   }
 };
 constexpr int kTmapCache = 64;
@@ -954,8 +1023,8 @@ struct TmapCache {
 };
 TmapCache g_tmaps;
 
-bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows) {
-  const TmapKey k{base, rows, cols, ld, box_rows};
+bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, int box_rows, int box_kb) {
+  const TmapKey k{base, rows, cols, ld, box_rows, box_kb};
   std::lock_guard<std::mutex> lock(g_tmaps.mu);
   for (int i = 0; i < kTmapCache; ++i) {
     if (g_tmaps.used[i] && g_tmaps.key[i] == k) {
@@ -963,7 +1032,7 @@ bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, i
       return true;
     }
   }
-  if (!encode_tmap(map, base, rows, cols, ld, box_rows)) return false;
+  if (!encode_tmap(map, base, rows, cols, ld, box_rows, box_kb)) return false;
   const int i = g_tmaps.next;
   g_tmaps.next = (i + 1) % kTmapCache;
   g_tmaps.key[i] = k;
@@ -975,10 +1044,11 @@ bool make_tmap(CUtensorMap* map, const void* base, int rows, int cols, int ld, i
 struct Plan {
   int tok_tile, tok_tiles, n_tiles;
   int ks;       // k-blocks per stage of gemm_tc_kernel
+  bool tmem_a;  // dequantized A in tensor memory
   Sched sc;
   int w_stages, b_stages, a_stages;
   uint32_t w_slot_bytes, b_slot_bytes;
-  uint32_t acc_cols, tmem_alloc;
+  uint32_t acc_cols, tmem_alloc, a_col0;
   size_t smem;
   size_t partial_bytes, counter_bytes;
 };
@@ -999,11 +1069,14 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.tok_tiles = (m + 255) / 256;
     P.tok_tile = round_up((m + P.tok_tiles - 1) / P.tok_tiles, 16);
   }
-  // Decode-sized tiles on 4-bit weights: two k-blocks per shared-memory stage
-  // where K has an even number of k-blocks (measured fastest on the OPT-30B
-  // decode shapes; every benchmark shape has even K/64).
-  const bool dec = w_bits == 4 && P.tok_tile <= kDecodeMaxTok;
-  P.ks = dec && kb_real % 2 == 0 ? 2 : 1;
+  // Decode-sized tiles move several k-blocks per copy (a copying thread
+  // completes about one copy per round trip, so bytes per copy set the rate):
+  // 4-bit weights four where the dequantized A ring still fits tensor memory
+  // with four k-blocks per slot (tokens <= 128), else two; fp16 weights two.
+  const bool dec = P.tok_tile <= kDecodeMaxTok;
+  if (dec && w_bits == 4 && P.tok_tile <= 128 && kb_real % 4 == 0) P.ks = 4;
+  else if (dec && kb_real % 2 == 0) P.ks = 2;
+  else P.ks = 1;
   const int kb_total = kb_real / P.ks;  // k-steps per tile
   const int min_iters = max(1, kMinItersPerCta / P.ks);
   P.n_tiles = (n + 127) / 128;
@@ -1045,19 +1118,27 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   // the rate at which they arrive from HBM).  Three activation slots when
   // that still leaves room for at least 8 weight k-steps, else two.
   const int budget = kMaxSmem - 1024 - kBarrierBytes - kEpiStageBytes;
-  {
+  // Decode-sized 4-bit tiles keep the dequantized A in tensor memory after
+  // the two accumulator buffers (512 columns: 2 x round_up(tokens, 32) + A
+  // slots of 64 columns); larger tiles need the columns for accumulators.
+  P.tmem_a = dec && w_bits == 4 && P.ks >= 2;
+  if (P.tmem_a) {
+    P.acc_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
+    P.a_col0 = 2 * P.acc_cols;
+    P.tmem_alloc = 512;
+  } else {
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
     P.acc_cols = cols;
     P.tmem_alloc = 2 * cols;
   }
-  const int a_slot = w_bits == 4 ? P.ks * kATileBytes : 0;
-  P.a_stages = w_bits == 4 ? 2 : 0;
+  const int a_slot = w_bits == 4 && !P.tmem_a ? P.ks * kATileBytes : 0;
+  P.a_stages = w_bits != 4 ? 0 : P.tmem_a ? std::min(4, static_cast<int>((512 - P.a_col0) / (32 * P.ks))) : 2;
   P.w_slot_bytes = static_cast<uint32_t>(w_bits == 4 ? round_up(P.ks * kTileBytes, 1024) : P.ks * kATileBytes);
   P.b_slot_bytes = static_cast<uint32_t>(P.ks * P.tok_tile * 128);
   const int rest = budget - P.a_stages * a_slot;
   const int w_slot = static_cast<int>(P.w_slot_bytes), b_slot = static_cast<int>(P.b_slot_bytes);
-  P.b_stages = rest - 3 * b_slot >= 8 * w_slot ? 3 : 2;
+  P.b_stages = rest - 3 * b_slot >= 4 * w_slot ? 3 : 2;
   P.w_stages = min(kMaxWStages, (rest - P.b_stages * b_slot) / w_slot);
   P.smem = static_cast<size_t>(P.a_stages) * a_slot + static_cast<size_t>(P.w_stages) * w_slot +
            static_cast<size_t>(P.b_stages) * b_slot + 1024 + kBarrierBytes + kEpiStageBytes;
@@ -1078,13 +1159,13 @@ cudaError_t configure_once() {
 
 // A fused LayerNorm needs every CTA resident at once (grid barrier), so that
 // variant is a cooperative launch; the grid never exceeds one CTA per SM.
-template <bool kW4, int KS>
+template <bool kW4, int KS, bool kTA>
 cudaError_t launch_general(const Plan& P, const CUtensorMap& tx, const CUtensorMap& tw, const GemmParams& p,
                            cudaStream_t s) {
-  const cudaError_t e = configure_once<gemm_tc_kernel<kW4, KS>>();
+  const cudaError_t e = configure_once<gemm_tc_kernel<kW4, KS, kTA>>();
   if (e != cudaSuccess) return e;
   if (!p.ln_on) {
-    gemm_tc_kernel<kW4, KS><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
+    gemm_tc_kernel<kW4, KS, kTA><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
     return launched();
   }
   cudaLaunchConfig_t cfg = {};
@@ -1097,7 +1178,7 @@ cudaError_t launch_general(const Plan& P, const CUtensorMap& tx, const CUtensorM
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<kW4, KS>, tx, tw, p);
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<kW4, KS, kTA>, tx, tw, p);
   if (le != cudaSuccess) return le;
   return launched();
 }
@@ -1129,10 +1210,10 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   const int n_bars = 2 * (P.w_stages + P.b_stages + P.a_stages) + 5;
   if (n_bars > kMaxBarriers) return cudaErrorInvalidValue;
   CUtensorMap tx, tw;
-  if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile)) return cudaErrorInvalidValue;
+  if (!make_tmap(&tx, a.x, a.m, a.k, a.ldx, P.tok_tile, P.ks)) return cudaErrorInvalidValue;
   if (w4) {
     tw = tx;
-  } else if (!make_tmap(&tw, a.w, a.n, a.k, a.k, 128)) {
+  } else if (!make_tmap(&tw, a.w, a.n, a.k, a.k, 128, P.ks)) {
     return cudaErrorInvalidValue;
   }
   GemmParams p{};
@@ -1149,6 +1230,7 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.b_slot_bytes = P.b_slot_bytes;
   p.acc_cols = P.acc_cols;
   p.tmem_alloc = P.tmem_alloc;
+  p.a_col0 = P.a_col0;
   p.sc = P.sc;
   p.bias = a.bias;
   p.residual = a.residual;
@@ -1192,9 +1274,13 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
     p.ln_on = 1;
     p.ln = *a.ln;
   }
-  if (w4 && P.ks == 2) return launch_general<true, 2>(P, tx, tw, p, s);
-  if (w4) return launch_general<true, 1>(P, tx, tw, p, s);
-  return launch_general<false, 1>(P, tx, tw, p, s);
+  if (w4 && P.tmem_a) {
+    if (P.ks == 4) return launch_general<true, 4, true>(P, tx, tw, p, s);
+    return launch_general<true, 2, true>(P, tx, tw, p, s);
+  }
+  if (w4) return launch_general<true, 1, false>(P, tx, tw, p, s);
+  if (P.ks == 2) return launch_general<false, 2, false>(P, tx, tw, p, s);
+  return launch_general<false, 1, false>(P, tx, tw, p, s);
 }
 
 }  // namespace flexq
