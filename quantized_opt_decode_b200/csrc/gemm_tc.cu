@@ -55,11 +55,12 @@
 namespace flexq {
 namespace {
 
-constexpr int kThreads = 480;  // 15 warps: W producer, MMA, 8 dequantizing, 4 epilogue, B producer
+constexpr int kThreads = 512;  // 16 warps: W producer, MMA, 8 dequantizing, 4 epilogue, B producer, MMA
 constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
 constexpr int kBWarp = 14;
+constexpr int kMma2Warp = 15;  // second MMA-issuing warp (odd k-blocks of a step)
 constexpr int kATileBytes = 128 * 64 * 2;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
@@ -89,7 +90,10 @@ struct GemmParams {
   int kb_real;  // 64-wide k-blocks of K
   int w_stages, b_stages, a_stages;     // ring depths: weights, activations, dequantized A
   uint32_t w_slot_bytes, b_slot_bytes;
-  uint32_t acc_cols;    // TMEM columns between the two accumulator buffers
+  uint32_t acc_cols;    // TMEM columns between accumulator buffers
+  uint32_t chain_cols;  // TMEM columns between the two issuers' accumulators of a buffer
+  int issuers;          // MMA-issuing threads (k-blocks alternate between them)
+  int acc_bufs;         // accumulator buffers (2: the epilogue overlaps the next segment)
   uint32_t tmem_alloc;  // columns allocated (power of two)
   uint32_t a_col0;      // first TMEM column of the dequantized A ring (A in tensor memory)
   Sched sc;
@@ -294,9 +298,14 @@ __device__ __forceinline__ void store_row16(const GemmParams& p, float (&v)[16],
 }
 
 // Accumulator buffer and phase parity used by segment q.
-__device__ __forceinline__ void acc_slot(int q, int& buf, uint32_t& parity) {
-  buf = q & 1;
-  parity = static_cast<uint32_t>(q >> 1) & 1u;
+__device__ __forceinline__ void acc_slot(int q, int bufs, int& buf, uint32_t& parity) {
+  if (bufs == 2) {
+    buf = q & 1;
+    parity = static_cast<uint32_t>(q >> 1) & 1u;
+  } else {
+    buf = 0;
+    parity = static_cast<uint32_t>(q) & 1u;
+  }
 }
 
 // Shared-memory words of the epilogue and the teardown, after the rings.
@@ -342,6 +351,24 @@ __device__ __forceinline__ bool wait_counter(const int* ctr, int target, uint64_
 // ---------------------------------------------------------------------------
 // epilogue role (warps kEpiWarp0 .. kEpiWarp0 + 3)
 // ---------------------------------------------------------------------------
+// 16 accumulator columns (tokens col .. col + 15) of this thread's TMEM lane:
+// the sum of the issuers' accumulators, in issuer order.  Warp-wide.
+__device__ __forceinline__ void acc_load16(const GemmParams& p, uint32_t tbase, uint32_t col, float (&v)[16]) {
+  uint32_t rr[16];
+  __syncwarp();
+  tmem_ld_x16(tbase + col, rr);
+  tmem_ld_wait();
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]);
+  if (p.issuers > 1) {
+    __syncwarp();
+    tmem_ld_x16(tbase + p.chain_cols + col, rr);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(rr[j]);
+  }
+}
+
 __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_base, int warp, int lane) {
   const Sched& sc = p.sc;
   const int cta = blockIdx.x;
@@ -354,7 +381,7 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
   for (int q = 0; get_seg(sc, cta, q, g); ++q) {
     int buf;
     uint32_t par;
-    acc_slot(q, buf, par);
+    acc_slot(q, p.acc_bufs, buf, par);
     const bool ok = mbar_wait(&c.accf[buf], par, drain_ns(p.wait_ns));
     if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
     tc_fence_after();
@@ -404,12 +431,10 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
         // consecutive features of one token)
         float* slot = p.partials + static_cast<size_t>(g.slot) * p.tok_tile * 128;
         for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
-          uint32_t rr[16];
-          __syncwarp();
-          tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
-          tmem_ld_wait();
+          float a[16];
+          acc_load16(p, tbase, static_cast<uint32_t>(c0), a);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(slot + (c0 + j) * 128 + frow, __uint_as_float(rr[j]));
+          for (int j = 0; j < 16; ++j) __stcg(slot + (c0 + j) * 128 + frow, a[j]);
         }
         tc_fence_before();
         mbar_arrive(&c.acce[buf]);
@@ -435,9 +460,7 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       for (int j = 0; j < 16; ++j) nxt[j] = __ldcg(other + j * 128 + frow);
     }
     for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
-      uint32_t rr[16];
-      __syncwarp();
-      tmem_ld_x16(tbase + static_cast<uint32_t>(c0), rr);
+      float acc[16];
       float v[16];
       if (one_other) {
         float cur[16];
@@ -447,20 +470,17 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
 #pragma unroll
           for (int j = 0; j < 16; ++j) nxt[j] = __ldcg(other + (c0 + 16 + j) * 128 + frow);
         }
-        tmem_ld_wait();
+        acc_load16(p, tbase, static_cast<uint32_t>(c0), acc);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float a = __uint_as_float(rr[j]);
-          v[j] = me == 0 ? (0.f + a) + cur[j] : (0.f + cur[j]) + a;
-        }
+        for (int j = 0; j < 16; ++j) v[j] = me == 0 ? (0.f + acc[j]) + cur[j] : (0.f + cur[j]) + acc[j];
       } else if (!g.full) {
-        tmem_ld_wait();
+        acc_load16(p, tbase, static_cast<uint32_t>(c0), acc);
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.f;
         for (int k = 0; k < ns; ++k) {
           if (k == me) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] += __uint_as_float(rr[j]);
+            for (int j = 0; j < 16; ++j) v[j] += acc[j];
           } else {
             const float* src = p.partials + static_cast<size_t>(c.fin_slots[k]) * p.tok_tile * 128;
             float t[16];
@@ -471,9 +491,7 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
           }
         }
       } else {
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(rr[j]);
+        acc_load16(p, tbase, static_cast<uint32_t>(c0), v);
       }
       // transpose 32 features x 16 tokens through shared memory so each lane
       // finishes 16 consecutive features of one token
@@ -708,21 +726,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t b_bytes = static_cast<uint32_t>(p.tok_tile) * 128u;  // one 64-wide activation box
 
   if (threadIdx.x == 0) {
+    // barriers the MMA issuers commit to count one arrival per issuer
     for (int s = 0; s < SW; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], kW4 ? kDequantThreads : 1);
+      mbar_init(&wempty[s], kW4 ? kDequantThreads : p.issuers);
     }
     for (int s = 0; s < SB; ++s) {
       mbar_init(&bfull[s], 1);
-      mbar_init(&bempty[s], 1);
+      mbar_init(&bempty[s], p.issuers);
     }
     for (int s = 0; s < SA; ++s) {
       mbar_init(&afull[s], kDequantThreads);
-      mbar_init(&aempty[s], 1);
+      mbar_init(&aempty[s], p.issuers);
     }
-    mbar_init(drained, 1);
+    mbar_init(drained, p.issuers);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&c.accf[b], 1);
+      mbar_init(&c.accf[b], p.issuers);
       mbar_init(&c.acce[b], kEpiThreads);
     }
     *c.abort_flag = 0;
@@ -786,9 +805,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, n - S); j < n; ++j)
         mbar_wait(&full[j % S], static_cast<uint32_t>(j / S) & 1u, drain_ns(p.wait_ns));
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp == 1 || warp == kMma2Warp) {
+    // ------------------------------------------------------------ MMA issuers
+    // One issuing thread completes about one tcgen05.mma per ~120 cycles
+    // whatever N, so decode tiles use two (warps 1 and 15): issuer mi takes
+    // the k-blocks u of a step with u % issuers == mi into its own
+    // accumulator (chain_cols apart); the epilogue adds the two.
+    const int mi = warp == 1 ? 0 : 1;
+    if (lane == 0 && mi < p.issuers) {
       const uint32_t idesc = idesc_f16_m128(static_cast<uint32_t>(p.tok_tile));
       // descriptors of slot 0; a slot is reached by adding its byte offset >> 4
       const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(kW4 && !kTA ? a_ring : w_ring));
@@ -803,14 +827,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; get_seg(sc, cta, q, g); ++q) {
         int buf;
         uint32_t par;
-        acc_slot(q, buf, par);
+        acc_slot(q, p.acc_bufs, buf, par);
         if (!stop && !mbar_wait(&c.acce[buf], par ^ 1u, p.wait_ns)) {
           set_error(p.err, DEV_TIMEOUT_MMA);
           *c.abort_flag = 1;
         }
         if (*c.abort_flag) stop = true;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * p.acc_cols;
+        const uint32_t d_tmem =
+            tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + static_cast<uint32_t>(mi) * p.chain_cols;
         for (int ks = g.kb0; ks < g.kb1 && !stop; ++ks, rb.next(SB), ra.next(SAx)) {
           bool ok = kW4 ? mbar_wait(&afull[ra.s], ra.ph, p.wait_ns) : mbar_wait(&wfull[ra.s], ra.ph, p.wait_ns);
           ok = ok && mbar_wait(&bfull[rb.s], rb.ph, p.wait_ns);
@@ -828,18 +853,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t a_tmem = a_tmem0 + static_cast<uint32_t>(ra.s * KS * 32);
 #pragma unroll
             for (int u = 0; u < KS; ++u)
+              if (u % p.issuers == mi) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ts(d_tmem, a_tmem + u * 32 + 8 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk, idesc,
-                           (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_f16_ts(d_tmem, a_tmem + u * 32 + 8 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk, idesc,
+                             (ks > g.kb0 || u >= p.issuers || kk > 0) ? 1u : 0u);
+              }
           } else {
             const uint64_t adesc = adesc0 + static_cast<uint64_t>(ra.s * a_step);
 #pragma unroll
             for (int u = 0; u < KS; ++u)
+              if (u % p.issuers == mi) {
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_f16_ss(d_tmem, adesc + u * (kATileBytes >> 4) + 2 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk,
-                           idesc, (ks > g.kb0 || u > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_f16_ss(d_tmem, adesc + u * (kATileBytes >> 4) + 2 * kk, bdesc + u * (b_bytes >> 4) + 2 * kk,
+                             idesc, (ks > g.kb0 || u >= p.issuers || kk > 0) ? 1u : 0u);
+              }
           }
           mma_commit(&bempty[rb.s]);
           mma_commit(kW4 ? &aempty[ra.s] : &wempty[ra.s]);
@@ -1048,7 +1077,8 @@ struct Plan {
   Sched sc;
   int w_stages, b_stages, a_stages;
   uint32_t w_slot_bytes, b_slot_bytes;
-  uint32_t acc_cols, tmem_alloc, a_col0;
+  uint32_t acc_cols, chain_cols, tmem_alloc, a_col0;
+  int issuers, acc_bufs;
   size_t smem;
   size_t partial_bytes, counter_bytes;
 };
@@ -1121,15 +1151,24 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   // Decode-sized 4-bit tiles keep the dequantized A in tensor memory after
   // the two accumulator buffers (512 columns: 2 x round_up(tokens, 32) + A
   // slots of 64 columns); larger tiles need the columns for accumulators.
+  // Tensor memory (512 columns) for 4-bit decode tiles: two issuers'
+  // accumulators per buffer, two buffers where they fit with two A slots
+  // (tokens <= 64), else one, then the A ring.
   P.tmem_a = dec && w_bits == 4 && P.ks >= 2;
   if (P.tmem_a) {
-    P.acc_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
-    P.a_col0 = 2 * P.acc_cols;
+    P.issuers = 2;
+    P.chain_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
+    P.acc_cols = 2 * P.chain_cols;
+    P.acc_bufs = 2 * P.acc_cols + 2u * 32u * P.ks <= 512u ? 2 : 1;
+    P.a_col0 = static_cast<uint32_t>(P.acc_bufs) * P.acc_cols;
     P.tmem_alloc = 512;
   } else {
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(P.tok_tile)) cols <<= 1;
+    P.issuers = 1;
+    P.chain_cols = cols;
     P.acc_cols = cols;
+    P.acc_bufs = 2;
     P.tmem_alloc = 2 * cols;
   }
   const int a_slot = w_bits == 4 && !P.tmem_a ? P.ks * kATileBytes : 0;
@@ -1229,6 +1268,9 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   p.w_slot_bytes = P.w_slot_bytes;
   p.b_slot_bytes = P.b_slot_bytes;
   p.acc_cols = P.acc_cols;
+  p.chain_cols = P.chain_cols;
+  p.issuers = P.issuers;
+  p.acc_bufs = P.acc_bufs;
   p.tmem_alloc = P.tmem_alloc;
   p.a_col0 = P.a_col0;
   p.sc = P.sc;
