@@ -60,7 +60,7 @@ constexpr int kDequantThreads = 256;
 constexpr int kEpiThreads = 128;
 constexpr int kEpiWarp0 = 10;
 constexpr int kBWarp = 14;
-constexpr int kMma2Warp = 15;  // second MMA-issuing warp (odd k-blocks of a step)
+constexpr int kMmaWarp2 = 15;  // second MMA-issuing warp (issuer 0 is warp 1)
 constexpr int kATileBytes = 128 * 64 * 2;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
@@ -91,8 +91,8 @@ struct GemmParams {
   int w_stages, b_stages, a_stages;     // ring depths: weights, activations, dequantized A
   uint32_t w_slot_bytes, b_slot_bytes;
   uint32_t acc_cols;    // TMEM columns between accumulator buffers
-  uint32_t chain_cols;  // TMEM columns between the two issuers' accumulators of a buffer
-  int issuers;          // MMA-issuing threads (k-blocks alternate between them)
+  uint32_t chain_cols;  // TMEM columns between the issuers' accumulators of a buffer
+  int issuers;          // MMA-issuing threads, 1, 2 or 4 (k-blocks of a step round-robin)
   int acc_bufs;         // accumulator buffers (2: the epilogue overlaps the next segment)
   uint32_t tmem_alloc;  // columns allocated (power of two)
   uint32_t a_col0;      // first TMEM column of the dequantized A ring (A in tensor memory)
@@ -160,16 +160,25 @@ __device__ __forceinline__ bool get_seg(const Sched& s, int c, int q, Seg& g) {
     g.slot = c;
     return g.kb1 > g.kb0;
   }
+  // The CTA's iterations [it0, it1) touch tiles t0 .. t1; its first and last
+  // tiles may be partial (shared with the neighbouring CTAs).  Partial
+  // segments run first, then the whole tiles: a split tile's contributors
+  // then all finish it early, its fixup overlaps the whole tiles, and the
+  // kernel ends on plain epilogues rather than on waits for partners.
   const long long it0 = sk_start(s, c), it1 = sk_start(s, c + 1);
-  long long it = it0;
-  for (int i = 0; i < q && it < it1; ++i) it = (it / s.kb_total + 1) * s.kb_total;
-  if (it >= it1) return false;
-  g.tile = static_cast<int>(it / s.kb_total);
-  g.kb0 = static_cast<int>(it % s.kb_total);
+  if (it1 <= it0) return false;
+  const long long t0 = it0 / s.kb_total, t1 = (it1 - 1) / s.kb_total;
+  const int n_seg = static_cast<int>(t1 - t0 + 1);
+  if (q >= n_seg) return false;
+  const bool last_part = it1 % s.kb_total != 0 && n_seg > 1;
+  const int i = !last_part ? q : q == 0 ? n_seg - 1 : q - 1;  // index in iteration order
+  const long long it = i == 0 ? it0 : (t0 + i) * s.kb_total;
+  g.tile = static_cast<int>(t0 + i);
+  g.kb0 = static_cast<int>(it - static_cast<long long>(g.tile) * s.kb_total);
   const long long end = min(it1, static_cast<long long>(g.tile + 1) * s.kb_total);
   g.kb1 = static_cast<int>(end - static_cast<long long>(g.tile) * s.kb_total);
   g.full = g.kb0 == 0 && g.kb1 == s.kb_total;
-  g.slot = 2 * c + (q == 0 ? 0 : 1);
+  g.slot = 2 * c + (i == 0 ? 0 : 1);
   return true;
 }
 
@@ -624,7 +633,7 @@ __device__ void ln_phase(const GemmParams& p, const Ctl& c) {
         }
       }
     }
-    const float var = block_sum_all(sq, red + 16) / static_cast<float>(p.n);
+    const float var = block_sum_all(sq, red + 32) / static_cast<float>(p.n);
     const float rstd = 1.0f / sqrtf(var + p.ln.eps);
     uint4* yr = reinterpret_cast<uint4*>(p.ln.y + static_cast<size_t>(r) * p.ln.ldy);
 #pragma unroll
@@ -805,7 +814,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = max(0, n - S); j < n; ++j)
         mbar_wait(&full[j % S], static_cast<uint32_t>(j / S) & 1u, drain_ns(p.wait_ns));
     }
-  } else if (warp == 1 || warp == kMma2Warp) {
+  } else if (warp == 1 || warp == kMmaWarp2) {
     // ------------------------------------------------------------ MMA issuers
     // One issuing thread completes about one tcgen05.mma per ~120 cycles
     // whatever N, so decode tiles use two (warps 1 and 15): issuer mi takes
@@ -1140,6 +1149,20 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     const long long per_cta = s.iters / s.grid;
     if ((kb_total + per_cta - 1) / per_cta + 1 > kMaxContrib)
       s.grid = static_cast<int>(std::max<long long>(1, s.iters * (kMaxContrib - 2) / kb_total));
+    // Few tiles (at most half as many as SMs): exactly two CTAs per tile (each
+    // half its k-steps) may finish sooner than spreading over every SM, since
+    // a tile with c contributors ends with the finalizer reading the others'
+    // partials, one L2 round trip (~1.5 k-steps, measured) per 16-token chunk
+    // and pair of contributors, while two contributors take the prefetched
+    // path.  Estimated in k-steps.
+    if (2 * tiles <= s.grid && kb_total % 2 == 0) {
+      const double per_all = static_cast<double>(s.iters) / s.grid;
+      const int contrib_all = static_cast<int>((kb_total + per_all - 1) / per_all) + 1;
+      const double chunks = P.tok_tile / 16.0;
+      const double cost_all = per_all + ((contrib_all - 1 + 1) / 2) * chunks * 1.5;
+      const double cost_two = kb_total / 2.0 + 0.2 * chunks;
+      if (cost_two < cost_all) s.grid = 2 * tiles;
+    }
     P.partial_bytes = static_cast<size_t>(2) * s.grid * tile_bytes;
   }
   if (P.partial_bytes > 0) P.counter_bytes = static_cast<size_t>(tiles) * 2 * sizeof(int);
@@ -1151,14 +1174,14 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
   // Decode-sized 4-bit tiles keep the dequantized A in tensor memory after
   // the two accumulator buffers (512 columns: 2 x round_up(tokens, 32) + A
   // slots of 64 columns); larger tiles need the columns for accumulators.
-  // Tensor memory (512 columns) for 4-bit decode tiles: two issuers'
+  // Tensor memory (512 columns) for 4-bit decode tiles: the two issuers'
   // accumulators per buffer, two buffers where they fit with two A slots
   // (tokens <= 64), else one, then the A ring.
   P.tmem_a = dec && w_bits == 4 && P.ks >= 2;
   if (P.tmem_a) {
-    P.issuers = 2;
     P.chain_cols = static_cast<uint32_t>(round_up(P.tok_tile, 32));
-    P.acc_cols = 2 * P.chain_cols;
+    P.issuers = 2;
+    P.acc_cols = static_cast<uint32_t>(P.issuers) * P.chain_cols;
     P.acc_bufs = 2 * P.acc_cols + 2u * 32u * P.ks <= 512u ? 2 : 1;
     P.a_col0 = static_cast<uint32_t>(P.acc_bufs) * P.acc_cols;
     P.tmem_alloc = 512;
