@@ -40,7 +40,13 @@ reason in the design notes):
   fp16 input.  Every other step stays float64.  A quantization decision is a
   step function of its input, so where a layer output hangs on those codes the
   oracle must take them from the input a fp16 layer sees; the GPU parity tests
-  therefore turn the option on for every shape.
+  therefore turn the option on for every shape;
+* ``Config.prefill_kv_cache`` (off by default): prefill attention reads the
+  pass's K/V back from the cache as stored (4-bit: quantized and dequantized,
+  fp16 mode: rounded to fp16) instead of using them as computed, i.e. it
+  consumes the compressed cache like the decode steps do ("FlexGen研究学术报告"
+  section 三(C): the KV cache is stored compressed and dequantized before
+  compute).
 Linear weights are stored [N_out][K_in], so a linear layer is y = x W^T + b.
 """
 from __future__ import annotations
@@ -68,6 +74,7 @@ class Config:
     ln1_f16: bool = False
     topk_permille: int = 0  # decode attention keeps the top ceil(L * permille / 1000) keys (0: dense)
     embed_bits: int = 16    # 4: the tied embedding E is stored group-wise 4-bit (groups along h)
+    prefill_kv_cache: bool = False  # prefill attention reads K/V back from the cache as stored
 
     @property
     def d(self) -> int:
@@ -78,7 +85,8 @@ class Config:
         return Config(layers=p["layers"], h=p["h"], heads=p["heads"], ffn=p["ffn"],
                       vocab=p["vocab"], w_bits=p["w_bits"], kv_bits=p["kv_bits"],
                       ln1_f16=ln1_f16, topk_permille=p.get("topk_permille", 0),
-                      embed_bits=p.get("embed_bits", 16))
+                      embed_bits=p.get("embed_bits", 16),
+                      prefill_kv_cache=bool(p.get("prefill_kv_cache", False)))
 
 
 # ---------------------------------------------------------------------------
@@ -302,6 +310,16 @@ def _mlp(cfg, W, x_out):
     return linear(g, W["w_fc2"], W["b_fc2"]) + x_out
 
 
+def cached_rows(cfg: Config, x: np.ndarray) -> np.ndarray:
+    """The values the cache returns for rows x [..., h] once stored: fp16
+    rounding, then (4-bit mode) the codec's round trip on 64-element groups
+    along h, which are the per-head groups of the cache since d % 64 == 0."""
+    x16 = np.asarray(x, dtype=np.float64).astype(np.float16)
+    if cfg.kv_bits == 4:
+        return q64.roundtrip(x16).astype(np.float64)
+    return x16.astype(np.float64)
+
+
 def layer_prefill(cfg: Config, W: dict, x: np.ndarray):
     """x: [b, s, h] -> (y [b, s, h], K16 [b, s, h], V16 [b, s, h]).  K16/V16
     are the fp16-rounded keys/values the cache stores for slots 0..s-1."""
@@ -310,7 +328,8 @@ def layer_prefill(cfg: Config, W: dict, x: np.ndarray):
     qkv = linear(u, W["w_qkv"], W["b_qkv"])
     Q, K, V = qkv[..., :h], qkv[..., h:2 * h], qkv[..., 2 * h:]
     a = cfg.heads
-    o = heads_merge(attention_causal(heads_split(Q, a), heads_split(K, a), heads_split(V, a)))
+    Ka, Va = (cached_rows(cfg, K), cached_rows(cfg, V)) if cfg.prefill_kv_cache else (K, V)
+    o = heads_merge(attention_causal(heads_split(Q, a), heads_split(Ka, a), heads_split(Va, a)))
     x_out = linear(o, W["w_o"], W["b_o"]) + x
     y = _mlp(cfg, W, x_out)
     return y, K.astype(np.float16), V.astype(np.float16)

@@ -9,6 +9,7 @@ section "P/D阶段计算"; multi-head form: survey notes eqs. (1)-(3); sizes:
 section "内存占用分析" (parameter count l(12h^2+13h)+Vh, per-layer fp16 bytes
 8h1^2 + 4h1h2, peak KV 4blh(s+n)).
 """
+import dataclasses
 import math
 import os
 
@@ -573,3 +574,26 @@ def test_topk_attention_brute_force_and_limits(rng):
     for i in range(b):
         for j in range(a):
             assert np.allclose(one[i, j], p[i, j, top[i, j]] * v[i, j, top[i, j]], rtol=1e-13)
+
+
+@pytest.mark.parametrize("kv_bits", [4, 16])
+def test_prefill_reading_the_cache_equals_decode_steps(kv_bits):
+    """With prefill_kv_cache the prefill's row t equals a decode step of token
+    t over a cache holding rows 0..t-1: the decode path appends the token's
+    K/V and reads every slot back through KVCache (quantize_rows /
+    dequantize_rows in 4-bit mode), a different route from the prefill's
+    cached_rows round trip."""
+    cfg = dataclasses.replace(tiny_cfg(kv_bits=kv_bits), prefill_kv_cache=True)
+    W = rand_layer(cfg)
+    rng = np.random.default_rng(11)
+    s = 7
+    x = rng.standard_normal((2, s, cfg.h))
+    y, _, _ = opt.layer_prefill(cfg, W, x)
+    cache = opt.KVCache(cfg, 2, s, kv_bits)
+    for t in range(s):
+        yt = opt.layer_decode(cfg, W, x[:, t], cache, t)
+        assert np.allclose(yt, y[:, t], rtol=1e-9, atol=1e-9), t
+    # and the option matters in 4-bit mode (the pass's own K/V differ from the cache's)
+    y_plain, _, _ = opt.layer_prefill(dataclasses.replace(cfg, prefill_kv_cache=False), W, x)
+    if kv_bits == 4:
+        assert not np.allclose(y_plain, y, rtol=1e-6, atol=1e-6)
