@@ -195,6 +195,8 @@ def kernel_work(p: dict, kind: str, M: int, L_avg: float):
             return M * a * (L_avg + kept) * kvb + 2 * M * h * 2, 2.0 * M * (L_avg + kept) * h
         return M * a * L_avg * 2 * kvb + 2 * M * h * 2, 4.0 * M * L_avg * h
     if kind == "attn_prefill":  # causal: half of the s x s score and value products
+        if p.get("prefill_kv_cache"):  # Q and O fp16, K and V read back from the cache
+            return M * h * 2 * 2 + 2 * M * a * kvb, 2.0 * M * L_avg * h
         return M * h * 2 * 4, 2.0 * M * L_avg * h
     if kind == "kv_append":
         return M * 2 * h * 2 + M * a * 2 * kvb, 0.0
@@ -457,6 +459,10 @@ def workload_name(args) -> str:
         name += "+embed4"
     if args.topk:
         name += f"+topk{args.topk}"
+    if args.prefill_kv_cache:
+        name += "+prefillkv"
+    if args.no_launch_overlap:
+        name += "+nooverlap"
     return name
 
 
@@ -478,6 +484,7 @@ def run_flexq(args, p):
     build.build()
     from quantized_opt_decode_b200 import flexq as fq
     from quantized_opt_decode_b200.device_model import DeviceModel, workspace
+    fq.flexq_set_launch_overlap(not args.no_launch_overlap)
 
     b, s, n, gbs = p["b"], p["s"], p["n"], p["gpu_batch"]
     stream = torch.cuda.Stream()
@@ -602,6 +609,7 @@ def run_flexq(args, p):
                        "embed_bits": p.get("embed_bits", 16),
                        "attn": (f"top-k sparse, {p['topk_permille'] / 10:g} % of keys"
                                 if p.get("topk_permille") else "dense"),
+                       "prefill_kv": "read back from the cache" if p.get("prefill_kv_cache") else "the pass's own",
                        "parallelism": f"replicas x{world}",
                        "step": "decode phase: n-1 decode columns x all layers + LM head",
                        "l2": "no flush: inputs far larger than L2 (weights + KV per step)"},
@@ -660,6 +668,7 @@ def run_offload(args, p):
     build.build()
     from quantized_opt_decode_b200 import flexq as fq
     from quantized_opt_decode_b200.device_model import DeviceModel, workspace
+    fq.flexq_set_launch_overlap(not args.no_launch_overlap)
 
     s, n = p["s"], p["n"]
     stream, copy = torch.cuda.Stream(), torch.cuda.Stream()
@@ -750,6 +759,10 @@ def main():
                     help="4: tied embedding / LM head stored group-wise 4-bit")
     ap.add_argument("--topk", type=int, default=0,
                     help="top-k sparse decode attention keeping ceil(L * TOPK / 1000) keys (100 = 10 %%)")
+    ap.add_argument("--prefill-kv-cache", action="store_true",
+                    help="prefill attention reads K/V back from the (4-bit) cache")
+    ap.add_argument("--no-launch-overlap", action="store_true",
+                    help="launch every kernel after its predecessor completes (no programmatic dependent launch)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -758,6 +771,8 @@ def main():
         p["embed_bits"] = args.embed_bits
     if args.topk:
         p["topk_permille"] = args.topk
+    if args.prefill_kv_cache:
+        p["prefill_kv_cache"] = True
     if args.impl == "reference":
         run_reference(args, p)
     elif args.offload:

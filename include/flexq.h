@@ -68,6 +68,13 @@ flexq_status flexq_device_status(void* stream);
  * makes pipelined kernels give up and report FLEXQ_ERR_TIMEOUT. */
 flexq_status flexq_set_wait_limit_ns(uint64_t ns);
 
+/* Programmatic dependent launch of the GEMMs and the decode attention (on by
+ * default): such a kernel may start while its predecessor in the stream is
+ * still running; it streams weights at once and waits for the predecessor
+ * before touching anything earlier kernels write, so results are unchanged.
+ * Returns the previous setting; 0 turns the overlap off (for measurement). */
+int flexq_set_launch_overlap(int on);
+
 /* ------------------------------------------------------------------------ */
 /* Seeded synthetic inputs (not part of the method: workload generation).     */
 /* Element i of stream (seed, tensor_id) is splitmix64's output function      */
@@ -185,6 +192,11 @@ typedef struct {
   int attn_topk_permille; /* 0: dense decode attention; 1..1000: top-k sparse
                              decode attention keeping ceil(L * permille / 1000)
                              keys (100 = the pages' top 10 %); 4-bit KV only */
+  int prefill_kv_cache;   /* 0: prefill attention uses the pass's own fp16 K/V;
+                             1: it reads them back from the cache as stored
+                             (4-bit: the dequantized codes, "FlexGen研究学术报告"
+                             section 三(C): the cache is kept compressed and
+                             dequantized before compute) */
 } flexq_config;
 
 /* One decoder layer's parameters (device pointers).  Linear weights [N_out]
@@ -254,6 +266,16 @@ flexq_status flexq_attention_decode_topk(const flexq_config* cfg, const flexq_kv
 flexq_status flexq_attention_prefill(const flexq_config* cfg, const void* qkv_dev, int ldqkv,
                                      int b, int s, void* out_dev, int ldo, void* stream);
 
+/* Causal prefill attention whose keys and values are read back from the
+ * cache: q_dev fp16 [b*s][ldq] (Q of sequence i, token t at row i*s + t),
+ * query t attends over cache slots pos0 .. pos0 + t (stored by
+ * flexq_kv_append; 4-bit codes are dequantized as the codec does,
+ * fp16(fp32(code * scale) + min)).  pos0 + s <= kv->max_len; in 4-bit mode
+ * pos0 % 8 == 0.  out_dev fp16 [b*s][ldo]. */
+flexq_status flexq_attention_prefill_cache(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev,
+                                           int ldq, int b, int s, int pos0, void* out_dev, int ldo,
+                                           void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Layer steps ([WT] "P/D阶段计算", pre-LN OPT block).                          */
 /*   u = LN1(x); [Q|K|V] = u W_qkv^T + b_qkv; o = attention;                   */
@@ -267,7 +289,8 @@ size_t flexq_layer_workspace(const flexq_config* cfg, int rows, int mode);
 
 /* Prefill of one layer over b sequences of s tokens: x_dev, y_dev fp16
  * [b*s][h] (distinct).  Writes cache slots 0..s-1 (quantized in 4-bit
- * mode); attention uses the pass's own fp16 K/V. */
+ * mode); attention uses the pass's own fp16 K/V, or with
+ * cfg->prefill_kv_cache reads them back from those slots. */
 flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* layer,
                                  const void* x_dev, void* y_dev, const flexq_kv* kv, int b, int s,
                                  void* ws_dev, size_t ws_bytes, void* stream);

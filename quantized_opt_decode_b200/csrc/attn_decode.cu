@@ -100,6 +100,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 8) attn_decode_q4_kernel(const __half* __restrict__ q, int ldq, KvView kv,
                                                                   int heads, int len, __half* __restrict__ out,
                                                                   int ldo, float inv_sqrt_d, AppendRow app) {
+  pdl_wait();  // q, the cache and the outputs follow the stream's earlier kernels
   constexpr int DPL = D / 4;   // score pass: dimensions per lane (one group)
   constexpr int NW = DPL / 8;  // code words per lane per token
   constexpr int G = D / 64;    // groups per head row
@@ -446,6 +447,7 @@ __global__ void __launch_bounds__(kQ4Threads) attn_decode_q4_split_kernel(const 
                                                                     int ldo, float inv_sqrt_d, int span,
                                                                     float* __restrict__ part, int* __restrict__ ctr,
                                                                     uint64_t wait_ns, uint32_t* err) {
+  pdl_wait();  // q, the cache and the outputs follow the stream's earlier kernels
   using L = Q4Stage<D>;
   constexpr int G = L::G;
   constexpr int NS = L::stages;
@@ -707,9 +709,8 @@ cudaError_t launch_q4_dense(const __half* q, int ldq, const KvView& kv, int b, i
     if (e != cudaSuccess) return e;
   }
   dim3 grid(heads, b);
-  attn_decode_q4_kernel<D><<<grid, kThreads, smem, s>>>(q, ldq, kv, heads, len, out, ldo,
-                                                        1.0f / sqrtf(static_cast<float>(D)), app);
-  return launched();
+  return launch_pdl(attn_decode_q4_kernel<D>, grid, dim3(kThreads), smem, s, q, ldq, kv, heads, len, out, ldo,
+                    1.0f / sqrtf(static_cast<float>(D)), app);
 }
 
 template <int D>
@@ -723,10 +724,9 @@ cudaError_t launch_q4_split(const __half* q, int ldq, const KvView& kv, int b, i
   span = (span + kChunk - 1) / kChunk * kChunk;
   const int S = (len + span - 1) / span;
   dim3 grid(heads, b, S);
-  attn_decode_q4_split_kernel<D><<<grid, kQ4Threads, L::stages * L::bytes, s>>>(
-      q, ldq, kv, heads, len, out, ldo, 1.0f / sqrtf(static_cast<float>(D)), span, part, ctr,
-      runtime().wait_limit_ns, runtime().err);
-  return launched();
+  return launch_pdl(attn_decode_q4_split_kernel<D>, grid, dim3(kQ4Threads), L::stages * L::bytes, s, q, ldq, kv,
+                    heads, len, out, ldo, 1.0f / sqrtf(static_cast<float>(D)), span, part, ctr,
+                    runtime().wait_limit_ns, runtime().err);
 }
 
 // ---------------------------------------------------------------------------
@@ -748,6 +748,7 @@ __global__ void __launch_bounds__(kQ4Threads) attn_decode_f16_kernel(const __hal
                                                                      int ldo, float inv_sqrt_d, int span,
                                                                      float* __restrict__ part, int* __restrict__ ctr,
                                                                      uint64_t wait_ns, uint32_t* err) {
+  pdl_wait();  // q, the cache and the outputs follow the stream's earlier kernels
   using L = F16Stage<D>;
   constexpr int T = L::T, NS = L::stages;
   constexpr int TW = T / kComputeWarps;  // tokens per warp and chunk
@@ -909,10 +910,9 @@ cudaError_t launch_f16(const __half* q, int ldq, const KvView& kv, int b, int he
   span = (span + L::T - 1) / L::T * L::T;
   const int S = (len + span - 1) / span;
   dim3 grid(heads, b, S);
-  attn_decode_f16_kernel<D><<<grid, kQ4Threads, L::stages * L::bytes, s>>>(
-      q, ldq, kv, heads, len, out, ldo, 1.0f / sqrtf(static_cast<float>(D)), span, part, ctr,
-      runtime().wait_limit_ns, runtime().err);
-  return launched();
+  return launch_pdl(attn_decode_f16_kernel<D>, grid, dim3(kQ4Threads), L::stages * L::bytes, s, q, ldq, kv, heads,
+                    len, out, ldo, 1.0f / sqrtf(static_cast<float>(D)), span, part, ctr, runtime().wait_limit_ns,
+                    runtime().err);
 }
 
 }  // namespace

@@ -2,8 +2,12 @@
 //   x_out = softmax(x_Q x_K^T / sqrt(.)) x_V   (before W_O),
 // FlexGen walk-through section "P/D阶段计算" (prefill), per head as in the
 // survey notes' eq. (2), with the autoregressive (causal) mask: query i sees
-// keys 0..i.  The pass's K and V are used as computed (the cache keeps their
-// quantized copy for the decode steps).
+// keys 0..i.  By default the pass's K and V are used as computed (the cache
+// keeps their quantized copy for the decode steps); with the configuration's
+// prefill_kv_cache the K/V tiles are read back from the cache as stored
+// ("FlexGen研究学术报告" section 三(C): compressed cache, dequantized before
+// compute): fp16 rows of an fp16 cache, or 4-bit codes dequantized tile by tile
+// into shared memory (fp16(fp32(code * scale) + min), the codec's rounding).
 //
 // Flash-attention style: one CTA = 64 queries of one (sequence, head), 4 warps
 // x 16 query rows; K/V tiles of 64 keys double-buffered in shared memory with
@@ -74,27 +78,130 @@ __device__ __forceinline__ void load_tile(uint32_t sbase, const __half* g, int l
   }
 }
 
+// 4-bit cache tile of keys k0 .. k0 + 63 (cache slots pos0 + k0 ..) of head
+// row hr, dequantized into the swizzled [64][D] fp16 layout; rows past
+// `rows_valid` are zero.  K: one (key, 64-element group) per thread step;
+// V (token-interleaved words): one (8-token block, 8 dimensions) per step,
+// written as 8 rows of one 16-byte chunk.
+__device__ __forceinline__ __half dq16(uint32_t code, float sc, float mn) {
+  return __float2half_rn(__fadd_rn(__fmul_rn(static_cast<float>(code), sc), mn));
+}
+
 template <int D>
-__global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const __half* __restrict__ qkv, int ld, int seq,
-                                                                int heads, __half* __restrict__ out, int ldo,
-                                                                float scale_log2) {
+__device__ __forceinline__ void load_tile_q4(uint32_t sK, uint32_t sV, const KvView& kv, size_t hr, int pos0, int k0,
+                                             int rows_valid) {
+  constexpr int G = D / 64;
+  const uint8_t* kc = static_cast<const uint8_t*>(kv.k) + (hr * kv.max_len + pos0 + k0) * (D / 2);
+  const __half2* km = static_cast<const __half2*>(kv.k_meta) + (hr * kv.max_len + pos0 + k0) * G;
+  const __half2* vm = static_cast<const __half2*>(kv.v_meta) + (hr * kv.max_len + pos0 + k0) * G;
+  const uint32_t* vw = static_cast<const uint32_t*>(kv.v) + (hr * (kv_pad_len(kv.max_len) / 8) + (pos0 + k0) / 8) * D;
+  for (int idx = threadIdx.x; idx < 64 * G; idx += kThreads) {
+    const int r = idx / G, gg = idx % G;
+    uint4 out[8];
+    if (r < rows_valid) {
+      const uint4 c0 = *reinterpret_cast<const uint4*>(kc + r * (D / 2) + gg * 32);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(kc + r * (D / 2) + gg * 32 + 16);
+      const float2 ms = __half22float2(km[r * G + gg]);
+      const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        __half e[8];
+#pragma unroll
+        for (int n = 0; n < 8; ++n) e[n] = dq16((w[c] >> (4 * n)) & 0xFu, ms.y, ms.x);
+        out[c] = *reinterpret_cast<const uint4*>(e);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) out[c] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sK + swz<D>(r, gg * 8 + c)), "r"(out[c].x),
+                   "r"(out[c].y), "r"(out[c].z), "r"(out[c].w)
+                   : "memory");
+  }
+  for (int idx = threadIdx.x; idx < 8 * (D / 8); idx += kThreads) {
+    const int bi = idx / (D / 8), dc = idx % (D / 8);
+    const int gg = (dc * 8) / 64;
+    uint32_t w[8];
+    const bool any = bi * 8 < rows_valid;
+    if (any) {
+      const uint4 a = *reinterpret_cast<const uint4*>(vw + bi * D + dc * 8);
+      const uint4 b = *reinterpret_cast<const uint4*>(vw + bi * D + dc * 8 + 4);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int r = bi * 8 + kk;
+      uint4 o4 = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows_valid) {
+        const float2 ms = __half22float2(vm[r * G + gg]);
+        __half e[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) e[c] = dq16((w[c] >> (4 * kk)) & 0xFu, ms.y, ms.x);
+        o4 = *reinterpret_cast<const uint4*>(e);
+      }
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sV + swz<D>(r, dc)), "r"(o4.x), "r"(o4.y),
+                   "r"(o4.z), "r"(o4.w)
+                   : "memory");
+    }
+  }
+}
+
+// K/V source: kPass = the pass's rows in the Q/K/V buffer; kCache16 / kCache4
+// = the layer's cache (slots pos0 ..).
+enum PrefillKv : int { kPass = 0, kCache16 = 1, kCache4 = 2 };
+
+struct PrefillArgs {
+  const __half* q;  // row (sequence i, token t) at q + (i * seq + t) * ldq, head j at + j * D
+  int ldq;
+  const __half* k;  // kPass: K / V columns of the same buffer (ld = ldkv)
+  const __half* v;
+  int ldkv;
+  KvView kv;        // kCache16 / kCache4
+  int pos0;         // first cache slot of the pass (a multiple of 8 for kCache4)
+  int seq, heads;
+  __half* out;
+  int ldo;
+  float scale_log2;
+};
+
+template <int D, int KV>
+__global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sQ = smem_u32(smem);
   const uint32_t sK = sQ + BQ * D * 2;
   const uint32_t sV = sK + 2 * BK * D * 2;
   const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
   const int j = blockIdx.y, i = blockIdx.z;
-  const int h = heads * D;
-  const __half* base = qkv + static_cast<size_t>(i) * seq * ld;
-  const __half* gQ = base + j * D;
-  const __half* gK = base + h + j * D;
-  const __half* gV = base + 2 * h + j * D;
+  const int seq = a.seq;
+  const size_t hr = static_cast<size_t>(i) * a.heads + j;
+  const __half* gQ = a.q + static_cast<size_t>(i) * seq * a.ldq + j * D;
+  const __half* gK;
+  const __half* gV;
+  int ldkv;
+  if (KV == kPass) {
+    gK = a.k + static_cast<size_t>(i) * seq * a.ldkv + j * D;
+    gV = a.v + static_cast<size_t>(i) * seq * a.ldkv + j * D;
+    ldkv = a.ldkv;
+  } else {
+    gK = static_cast<const __half*>(a.kv.k) + (hr * a.kv.max_len + a.pos0) * D;
+    gV = static_cast<const __half*>(a.kv.v) + (hr * a.kv.max_len + a.pos0) * D;
+    ldkv = D;
+  }
+  __half* out = a.out;
+  const int ldo = a.ldo;
+  const float scale_log2 = a.scale_log2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q0 = qb * BQ;
 
-  load_tile<D>(sQ, gQ, ld, q0, min(BQ, seq - q0));
-  load_tile<D>(sK, gK, ld, 0, min(BK, seq));
-  load_tile<D>(sV, gV, ld, 0, min(BK, seq));
+  load_tile<D>(sQ, gQ, a.ldq, q0, min(BQ, seq - q0));
+  if (KV == kCache4) {
+    load_tile_q4<D>(sK, sV, a.kv, hr, a.pos0, 0, min(BK, seq));
+  } else {
+    load_tile<D>(sK, gK, ldkv, 0, min(BK, seq));
+    load_tile<D>(sV, gV, ldkv, 0, min(BK, seq));
+  }
   cp_commit();
 
   float o[D / 8][4];
@@ -109,8 +216,13 @@ __global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const __half* __
     const int buf = kt & 1;
     if (kt + 1 < ntiles) {
       const int k0 = (kt + 1) * BK;
-      load_tile<D>(sK + (buf ^ 1) * BK * D * 2, gK, ld, k0, min(BK, seq - k0));
-      load_tile<D>(sV + (buf ^ 1) * BK * D * 2, gV, ld, k0, min(BK, seq - k0));
+      if (KV == kCache4) {
+        load_tile_q4<D>(sK + (buf ^ 1) * BK * D * 2, sV + (buf ^ 1) * BK * D * 2, a.kv, hr, a.pos0, k0,
+                        min(BK, seq - k0));
+      } else {
+        load_tile<D>(sK + (buf ^ 1) * BK * D * 2, gK, ldkv, k0, min(BK, seq - k0));
+        load_tile<D>(sV + (buf ^ 1) * BK * D * 2, gV, ldkv, k0, min(BK, seq - k0));
+      }
     }
     cp_commit();
     cp_wait<1>();
@@ -212,19 +324,21 @@ __global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const __half* __
   }
 }
 
-template <int D>
-cudaError_t launch_d(const __half* qkv, int ld, int b, int seq, int heads, __half* out, int ldo, cudaStream_t s) {
+template <int D, int KV>
+cudaError_t launch_d(PrefillArgs a, int b, cudaStream_t s) {
   const int smem = (BQ + 4 * BK) * D * 2;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  dim3 grid((seq + BQ - 1) / BQ, heads, b);
-  const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
-  attn_prefill_kernel<D><<<grid, kThreads, smem, s>>>(qkv, ld, seq, heads, out, ldo, scale_log2);
+  static const cudaError_t configured =
+      cudaFuncSetAttribute(attn_prefill_kernel<D, KV>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (configured != cudaSuccess) return configured;
+  dim3 grid((a.seq + BQ - 1) / BQ, a.heads, b);
+  a.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+  attn_prefill_kernel<D, KV><<<grid, kThreads, smem, s>>>(a);
   return launched();
+}
+
+template <int KV>
+cudaError_t launch_kv(const PrefillArgs& a, int b, int d, cudaStream_t s) {
+  return d == 128 ? launch_d<128, KV>(a, b, s) : launch_d<64, KV>(a, b, s);
 }
 
 }  // namespace
@@ -232,8 +346,33 @@ cudaError_t launch_d(const __half* qkv, int ld, int b, int seq, int heads, __hal
 cudaError_t launch_attn_prefill(const __half* qkv, int ldqkv, int b, int seq, int heads, int d, __half* out,
                                 int ldo, cudaStream_t s) {
   if (b == 0 || seq == 0) return cudaSuccess;
-  return d == 128 ? launch_d<128>(qkv, ldqkv, b, seq, heads, out, ldo, s)
-                  : launch_d<64>(qkv, ldqkv, b, seq, heads, out, ldo, s);
+  PrefillArgs a{};
+  a.q = qkv;
+  a.ldq = ldqkv;
+  a.k = qkv + heads * d;
+  a.v = qkv + 2 * heads * d;
+  a.ldkv = ldqkv;
+  a.seq = seq;
+  a.heads = heads;
+  a.out = out;
+  a.ldo = ldo;
+  return launch_kv<kPass>(a, b, d, s);
+}
+
+cudaError_t launch_attn_prefill_cache(const __half* q, int ldq, const KvView& kv, int kv_bits, int pos0, int b,
+                                      int seq, int heads, int d, __half* out, int ldo, cudaStream_t s) {
+  if (b == 0 || seq == 0) return cudaSuccess;
+  if (kv_bits == 4 && pos0 % 8 != 0) return cudaErrorInvalidValue;
+  PrefillArgs a{};
+  a.q = q;
+  a.ldq = ldq;
+  a.kv = kv;
+  a.pos0 = pos0;
+  a.seq = seq;
+  a.heads = heads;
+  a.out = out;
+  a.ldo = ldo;
+  return kv_bits == 4 ? launch_kv<kCache4>(a, b, d, s) : launch_kv<kCache16>(a, b, d, s);
 }
 
 }  // namespace flexq

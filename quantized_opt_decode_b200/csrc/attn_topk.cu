@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
                                                                   __half* __restrict__ out, int ldo,
                                                                   int32_t* __restrict__ idx_out,
                                                                   float inv_sqrt_d, AppendRow app) {
+  pdl_wait();  // q, the cache and the outputs follow the stream's earlier kernels
   constexpr int G = D / 64;
   constexpr int DPL = D / 4;
   constexpr int NW = DPL / 8;
@@ -408,9 +409,8 @@ cudaError_t launch_topk(const __half* q, int ldq, const KvView& kv, int b, int h
     if (e != cudaSuccess) return e;
   }
   dim3 grid(heads, b);
-  attn_topk_q4_kernel<D><<<grid, kTkThreads, smem, s>>>(q, ldq, kv, heads, len, kk, out, ldo, idx,
-                                                        1.0f / sqrtf(static_cast<float>(D)), app);
-  return launched();
+  return launch_pdl(attn_topk_q4_kernel<D>, grid, dim3(kTkThreads), smem, s, q, ldq, kv, heads, len, kk, out, ldo,
+                    idx, 1.0f / sqrtf(static_cast<float>(D)), app);
 }
 
 }  // namespace

@@ -198,6 +198,15 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while its predecessor in the
+// stream is still running; before its first access to memory that earlier
+// kernels write (activations, caches, workspaces) it waits for them with
+// pdl_wait().  Weights are never written by kernels and may be read before.
+// pdl_trigger() lets the successor launch before this kernel completes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // D[tmem] (+)= A[smem] * B[smem]^T, fp16 inputs, fp32 accumulation.
 __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {

@@ -25,6 +25,7 @@ namespace {
 
 thread_local std::string g_last_error;
 uint64_t g_wait_limit_ns = 2000000000ull;
+int g_pdl = 1;
 constexpr int kMaxDevices = 64;
 Runtime g_rt[kMaxDevices];
 std::once_flag g_rt_once[kMaxDevices];
@@ -115,6 +116,7 @@ flexq_status check_config(const flexq_config* c) {
   FQ_CHECK(c->ln_eps > 0.f, "ln_eps must be positive");
   FQ_CHECK(c->attn_topk_permille >= 0 && c->attn_topk_permille <= 1000, "attn_topk_permille must be in 0..1000");
   FQ_CHECK(c->attn_topk_permille == 0 || c->kv_bits == 4, "top-k sparse attention needs the 4-bit KV cache");
+  FQ_CHECK(c->prefill_kv_cache == 0 || c->prefill_kv_cache == 1, "prefill_kv_cache must be 0 or 1");
   return FLEXQ_OK;
 }
 
@@ -358,7 +360,11 @@ flexq_status layer_step(const flexq_config* c, const flexq_layer* L, const __hal
     FQ_CUDA(launch_kv_append(w.qkv + h, w.qkv + 2 * h, 3 * h, b, ntok, c->heads, d, c->kv_bits, kvv, pos, s),
             "KV append");
   }
-  if (prefill) {
+  if (prefill && c->prefill_kv_cache) {
+    ProfScope ps(FLEXQ_K_ATTN_PREFILL, s);
+    FQ_CUDA(launch_attn_prefill_cache(w.qkv, 3 * h, kvv, c->kv_bits, pos, b, ntok, c->heads, d, w.u, h, s),
+            "prefill attention (cache)");
+  } else if (prefill) {
     ProfScope ps(FLEXQ_K_ATTN_PREFILL, s);
     FQ_CUDA(launch_attn_prefill(w.qkv, 3 * h, b, ntok, c->heads, d, w.u, h, s), "prefill attention");
   } else {
@@ -406,6 +412,7 @@ const Runtime& runtime() {
     r.err = static_cast<uint32_t*>(p);
   });
   g_rt[dev].wait_limit_ns = g_wait_limit_ns;
+  g_rt[dev].pdl = g_pdl;
   return g_rt[dev];
 }
 
@@ -426,11 +433,17 @@ extern "C" {
 
 const char* flexq_last_error(void) { return g_last_error.c_str(); }
 
-int flexq_version(void) { return 101; }
+int flexq_version(void) { return 102; }
 
 flexq_status flexq_set_wait_limit_ns(uint64_t ns) {
   g_wait_limit_ns = ns == 0 ? 2000000000ull : ns;
   return FLEXQ_OK;
+}
+
+int flexq_set_launch_overlap(int on) {
+  const int old = g_pdl;
+  g_pdl = on ? 1 : 0;
+  return old;
 }
 
 flexq_status flexq_device_status(void* stream) {
@@ -654,6 +667,24 @@ flexq_status flexq_attention_prefill(const flexq_config* cfg, const void* qkv_de
   FQ_CUDA(launch_attn_prefill(static_cast<const __half*>(qkv_dev), ldqkv, b, s, cfg->heads, cfg->h / cfg->heads,
                               static_cast<__half*>(out_dev), ldo, as_stream(stream)),
           "prefill attention");
+  return FLEXQ_OK;
+}
+
+flexq_status flexq_attention_prefill_cache(const flexq_config* cfg, const flexq_kv* kv, const void* q_dev,
+                                           int ldq, int b, int s, int pos0, void* out_dev, int ldo, void* stream) {
+  FQ_TRY(check_config(cfg));
+  FQ_CHECK(b >= 0 && s >= 0 && pos0 >= 0, "b, s and pos0 must be >= 0");
+  if (b == 0 || s == 0) return FLEXQ_OK;
+  FQ_TRY(check_kv(cfg, kv, b));
+  FQ_CHECK(q_dev && out_dev, "NULL pointer");
+  FQ_CHECK(pos0 + s <= kv->max_len, "slots %d..%d exceed the cache (%d)", pos0, pos0 + s - 1, kv->max_len);
+  FQ_CHECK(cfg->kv_bits == 16 || pos0 % 8 == 0, "4-bit mode needs pos0 %% 8 == 0");
+  FQ_CHECK(ldq >= cfg->h && ldq % 8 == 0 && ldo >= cfg->h && ldo % 8 == 0, "bad row strides");
+  FQ_CHECK(aligned16(q_dev) && aligned16(out_dev), "pointers must be 16-byte aligned");
+  FQ_CUDA(launch_attn_prefill_cache(static_cast<const __half*>(q_dev), ldq, view_of(cfg, kv, 0), cfg->kv_bits, pos0,
+                                    b, s, cfg->heads, cfg->h / cfg->heads, static_cast<__half*>(out_dev), ldo,
+                                    as_stream(stream)),
+          "prefill attention (cache)");
   return FLEXQ_OK;
 }
 

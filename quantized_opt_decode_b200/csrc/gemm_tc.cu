@@ -379,6 +379,7 @@ __device__ __forceinline__ void acc_load16(const GemmParams& p, uint32_t tbase, 
 }
 
 __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_base, int warp, int lane) {
+  pdl_wait();  // the residual, outputs, partials and counters belong to the stream's order
   const Sched& sc = p.sc;
   const int cta = blockIdx.x;
   const int et = threadIdx.x - kEpiWarp0 * 32;
@@ -765,6 +766,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *c.tmem_slot;
   const Sched& sc = p.sc;
+  // The successor may launch now: its CTAs take SMs as this kernel's leave
+  // and stream their weights while these finish.
+  pdl_trigger();
 
   if (warp == 0 || warp == kBWarp) {
     // ------------------------------------------------------------ producers
@@ -775,6 +779,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // one 3-D tensor box of the activations or fp16 weights).
     if (lane == 0) {
       const bool w_role = warp == 0;
+      // weights are never written by kernels: only the activations wait for
+      // the predecessor
+      if (!w_role) pdl_wait();
       const uint64_t pol = w_role ? policy_evict_first() : policy_evict_last();
       if (w_role && !kW4) prefetch_tmap(&tmap_w);
       if (!w_role) prefetch_tmap(&tmap_x);
@@ -1226,10 +1233,7 @@ cudaError_t launch_general(const Plan& P, const CUtensorMap& tx, const CUtensorM
                            cudaStream_t s) {
   const cudaError_t e = configure_once<gemm_tc_kernel<kW4, KS, kTA>>();
   if (e != cudaSuccess) return e;
-  if (!p.ln_on) {
-    gemm_tc_kernel<kW4, KS, kTA><<<P.sc.grid, kThreads, P.smem, s>>>(tx, tw, p);
-    return launched();
-  }
+  if (!p.ln_on) return launch_pdl(gemm_tc_kernel<kW4, KS, kTA>, dim3(P.sc.grid), dim3(kThreads), P.smem, s, tx, tw, p);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P.sc.grid);
   cfg.blockDim = dim3(kThreads);

@@ -22,11 +22,34 @@ struct Runtime {
   uint64_t wait_limit_ns;  // deadline of every bounded device wait
   uint32_t* err;           // device error word
   int num_sms;
+  int pdl;                 // launch GEMMs and decode attention with programmatic dependent launch
 };
+
 const Runtime& runtime();
 
 // Counts one kernel launch of this library and returns the launch status.
 cudaError_t launched();
+
+// Launches `kernel` on `s`, with the programmatic stream-serialization
+// attribute when runtime().pdl (the kernel must pdl_wait() before touching
+// memory earlier kernels write), and counts it.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = runtime().pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+  if (e != cudaSuccess) return e;
+  return launched();
+}
 
 // Sets the calling thread's message returned by flexq_last_error().
 void set_last_error(const char* msg);
@@ -155,6 +178,10 @@ inline int topk_count(int len, int permille) {
 size_t attn_decode_partial_bytes(int b, int heads, int d);
 cudaError_t launch_attn_prefill(const __half* qkv, int ldqkv, int b, int seq, int heads, int d,
                                 __half* out, int ldo, cudaStream_t s);
+// Causal prefill attention of `seq` queries per sequence (q rows i * seq + t,
+// stride ldq) over cache slots pos0 .. pos0 + seq - 1 read back as stored.
+cudaError_t launch_attn_prefill_cache(const __half* q, int ldq, const KvView& kv, int kv_bits, int pos0, int b,
+                                      int seq, int heads, int d, __half* out, int ldo, cudaStream_t s);
 
 // embedding and greedy choice
 // E: fp16 [vocab][h] (embed_bits 16) or the 4-bit tiled layout (embed_bits 4).

@@ -21,7 +21,8 @@ LINEAR = ("w_qkv", "w_o", "w_fc1", "w_fc2")
 def make_config(p: dict) -> fq.flexq_config:
     return fq.flexq_config(h=p["h"], heads=p["heads"], ffn=p["ffn"], w_bits=p["w_bits"],
                            kv_bits=p["kv_bits"], ln_eps=1e-5,
-                           attn_topk_permille=p.get("topk_permille", 0))
+                           attn_topk_permille=p.get("topk_permille", 0),
+                           prefill_kv_cache=int(bool(p.get("prefill_kv_cache", False))))
 
 
 def fill_normal(t: torch.Tensor, seed: int, tid: int, sigma: float = 0.02, mean: float = 0.0,

@@ -41,7 +41,8 @@ VP = C.c_void_p
 
 class flexq_config(C.Structure):
     _fields_ = [("h", C.c_int), ("heads", C.c_int), ("ffn", C.c_int), ("w_bits", C.c_int),
-                ("kv_bits", C.c_int), ("ln_eps", C.c_float), ("attn_topk_permille", C.c_int)]
+                ("kv_bits", C.c_int), ("ln_eps", C.c_float), ("attn_topk_permille", C.c_int),
+                ("prefill_kv_cache", C.c_int)]
 
 
 class flexq_layer(C.Structure):
@@ -81,6 +82,7 @@ _SIGS = {
     "flexq_version": ([], C.c_int),
     "flexq_device_status": ([VP], C.c_int),
     "flexq_set_wait_limit_ns": ([C.c_uint64], C.c_int),
+    "flexq_set_launch_overlap": ([C.c_int], C.c_int),
     "flexq_synth_normal_f16": ([VP, C.c_size_t, C.c_uint64, C.c_uint64, C.c_size_t, C.c_float,
                                 C.c_float, VP], C.c_int),
     "flexq_synth_tokens": ([VP, C.c_size_t, C.c_uint64, C.c_uint64, C.c_size_t, C.c_int32, VP],
@@ -105,6 +107,8 @@ _SIGS = {
     "flexq_attention_decode_topk": ([_CFG, C.POINTER(flexq_kv), VP, C.c_int, C.c_int, C.c_int, C.c_int,
                                      VP, C.c_int, VP, VP], C.c_int),
     "flexq_attention_prefill": ([_CFG, VP, C.c_int, C.c_int, C.c_int, VP, C.c_int, VP], C.c_int),
+    "flexq_attention_prefill_cache": ([_CFG, C.POINTER(flexq_kv), VP, C.c_int, C.c_int, C.c_int, C.c_int, VP,
+                                       C.c_int, VP], C.c_int),
     "flexq_layer_workspace": ([_CFG, C.c_int, C.c_int], C.c_size_t),
     "flexq_layer_prefill": ([_CFG, C.POINTER(flexq_layer), VP, VP, C.POINTER(flexq_kv), C.c_int,
                              C.c_int, VP, C.c_size_t, VP], C.c_int),
@@ -171,6 +175,10 @@ def flexq_device_status(stream=None):
 
 def flexq_set_wait_limit_ns(ns: int):
     _check(_lib.flexq_set_wait_limit_ns(ns))
+
+
+def flexq_set_launch_overlap(on: bool) -> bool:
+    return bool(_lib.flexq_set_launch_overlap(1 if on else 0))
 
 
 def flexq_synth_normal_f16(out, n, seed, tensor_id, start=0, sigma=0.02, mean=0.0, stream=None):
@@ -246,6 +254,11 @@ def flexq_attention_decode_topk(cfg, kv, q, ldq, b, length, k, out, ldo, idx=Non
 def flexq_attention_prefill(cfg, qkv, ldqkv, b, s, out, ldo, stream=None):
     _check(_lib.flexq_attention_prefill(C.byref(cfg), _p(qkv), ldqkv, b, s, _p(out), ldo,
                                         _s(stream)))
+
+
+def flexq_attention_prefill_cache(cfg, kv, q, ldq, b, s, pos0, out, ldo, stream=None):
+    _check(_lib.flexq_attention_prefill_cache(C.byref(cfg), C.byref(kv), _p(q), ldq, b, s, pos0, _p(out),
+                                              ldo, _s(stream)))
 
 
 def flexq_layer_workspace(cfg, rows, mode) -> int:

@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(fq):
 
 
 def test_version_and_empty_error(fq):
-    assert fq.flexq_version() == 101
+    assert fq.flexq_version() == 102
 
 
 def _status(fn, *args):
@@ -71,7 +71,7 @@ def test_config_validation(fq):
     bad = [dict(h=100, heads=1), dict(h=256, heads=3), dict(h=256, heads=1),
            dict(h=256, heads=4, ffn=100), dict(h=256, heads=4, w_bits=8),
            dict(attn_topk_permille=1001), dict(attn_topk_permille=-1),
-           dict(kv_bits=16, attn_topk_permille=100)]
+           dict(kv_bits=16, attn_topk_permille=100), dict(prefill_kv_cache=2)]
     for over in bad:
         kw = dict(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=4, ln_eps=1e-5)
         kw.update(over)
@@ -154,3 +154,14 @@ def test_package_builds_from_scratch_and_binding_fails_loudly(tmp_path):
                        env=dict(os.environ, PYTHONPATH=str(tmp_path)))
     assert r.returncode == 0, r.stderr
     assert "refused:" in r.stdout and "libflexq.so" in r.stdout
+
+
+def test_prefill_cache_rejects_bad_arguments(fq):
+    cfg = fq.flexq_config(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=4, ln_eps=1e-5)
+    kv = fq.flexq_kv(0x1000, 0x2000, 0x3000, 0x4000, 4, 40)
+    st = fq._lib.flexq_attention_prefill_cache(C.byref(cfg), C.byref(kv), 0x1000, 256, 4, 36, 8, 0x2000, 256,
+                                               None)
+    assert st == 1 and "exceed" in fq.flexq_last_error()
+    st = fq._lib.flexq_attention_prefill_cache(C.byref(cfg), C.byref(kv), 0x1000, 256, 4, 16, 4, 0x2000, 256,
+                                               None)
+    assert st == 1 and "pos0" in fq.flexq_last_error()

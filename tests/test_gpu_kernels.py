@@ -180,6 +180,38 @@ def test_attention_prefill(h, heads, b, s):
     assert_close(to_host(out), ref, TOL, what=f"prefill attention s={s}")
 
 
+@pytest.mark.parametrize("h,heads,kv_bits,b,s,pos0", [(512, 4, 4, 2, 200, 0), (256, 4, 4, 3, 64, 0),
+                                                      (512, 4, 4, 2, 73, 8), (1024, 8, 4, 1, 130, 0),
+                                                      (512, 4, 16, 2, 130, 0), (256, 4, 16, 2, 37, 5)])
+def test_attention_prefill_from_cache(h, heads, kv_bits, b, s, pos0):
+    """Prefill attention reading K/V back from the cache: query t of the pass
+    attends over slots pos0 .. pos0 + t as stored (the oracle's KVCache
+    write/read, the decode steps' route), ragged last tiles included; slots
+    before pos0 hold other rows and must be ignored."""
+    cfg = _cfg(h, heads, kv_bits)
+    L = pos0 + s + 3
+    rng = np.random.default_rng(s + h + kv_bits + pos0)
+    rows = rng.standard_normal((b * s, 3 * h)).astype(np.float16)
+    early = rng.standard_normal((b * max(pos0, 1), 3 * h)).astype(np.float16) * 50
+    dev = _dev_cache(cfg, b, L)
+    rd = to_dev(rows)
+    if pos0 > 0:
+        ed = to_dev(early)
+        fq.flexq_kv_append(cfg, dev.struct, ed[:, h:], ed[:, 2 * h:], 3 * h, b, 0, pos0)
+    fq.flexq_kv_append(cfg, dev.struct, rd[:, h:], rd[:, 2 * h:], 3 * h, b, pos0, s)
+    out = torch.empty(b * s, h, dtype=torch.float16, device="cuda")
+    fq.flexq_attention_prefill_cache(cfg, dev.struct, rd, 3 * h, b, s, pos0, out, h)
+    fq.flexq_device_status()
+    ocfg = opt.Config(layers=1, h=h, heads=heads, ffn=4 * h, vocab=8, w_bits=4, kv_bits=kv_bits)
+    oc = opt.KVCache(ocfg, b, s, kv_bits)
+    r3 = rows.reshape(b, s, 3 * h)
+    oc.write("k", r3[..., h:2 * h], 0)
+    oc.write("v", r3[..., 2 * h:], 0)
+    Q = opt.heads_split(r3[..., :h].astype(np.float64), heads)
+    ref = opt.heads_merge(opt.attention_causal(Q, oc.read("k", s), oc.read("v", s))).reshape(b * s, h)
+    assert_close(to_host(out), ref, TOL, what=f"prefill attention from the {kv_bits}-bit cache s={s}")
+
+
 @pytest.mark.parametrize("h,heads,length,permille", [(512, 4, 545, 100), (256, 4, 37, 100), (1024, 8, 1030, 100),
                                                      (512, 4, 200, 1000), (256, 4, 64, 10), (512, 4, 1, 100)])
 def test_attention_decode_topk(h, heads, length, permille):

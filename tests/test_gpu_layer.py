@@ -74,6 +74,9 @@ def _check_out(got, ref, x):
     ("tiny16", {}),
     ("tiny", dict(h=512, heads=4, ffn=2048)),      # d = 128
     ("tiny16", dict(h=512, heads=4, ffn=2048)),
+    ("tiny", dict(prefill_kv_cache=True)),         # prefill attention reads the 4-bit cache back
+    ("tiny", dict(h=512, heads=4, ffn=2048, prefill_kv_cache=True)),
+    ("tiny16", dict(prefill_kv_cache=True)),
 ])
 def test_layer_prefill_and_decode(name, over):
     p = _preset(name, **over)
@@ -96,7 +99,8 @@ def test_layer_prefill_and_decode(name, over):
 
 @pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny16", {}),
                                        ("tiny", dict(embed_bits=4)),        # 4-bit tied embedding / LM head
-                                       ("tiny", dict(topk_permille=100))])  # top-10 % sparse decode attention
+                                       ("tiny", dict(topk_permille=100)),   # top-10 % sparse decode attention
+                                       ("tiny", dict(prefill_kv_cache=True))])  # prefill reads the 4-bit cache
 def test_generate_tokens_valid_under_oracle(name, over):
     p = _preset(name, **over)
     b, s, n = p["b"], p["s"], p["n"]
