@@ -50,10 +50,11 @@ __device__ __forceinline__ void load_words(const uint32_t* p, uint32_t (&w)[NW])
 // The V codes are token-interleaved (nibble k of word (block, dim) = token
 // 8*block + k), so dp4a weights 4 tokens of one dimension at a time:
 //   sum_t p_t x_hat_t,e = max_w/65535 * sum_t w_i,t code_t,e + sum_t p_t min_t.
-// Pass 1 (scores, four 16-byte loads in flight per lane), pass 2 (softmax
-// weights and their fixed-point packing), pass 3 (values, likewise four loads
-// in flight).  In a decode step warp 0 first appends the token's K/V rows to
-// the cache (quantize on append), so the step needs no separate launch.
+// Pass 1 (scores, six 16-byte loads in flight per lane), pass 2 (softmax
+// weights and their fixed-point packing), pass 3 (values, likewise six loads
+// in flight).  In a decode step the warps first append the token's K/V rows
+// to the cache (quantize on append, one warp per 64-element group), so the
+// step needs no separate launch.
 // ---------------------------------------------------------------------------
 constexpr int kThreads = 128;
 
@@ -70,7 +71,12 @@ __device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) 
 }
 
 constexpr int kStatN = 5;  // S, pm[2], wmax[2]
-constexpr int kUnroll = 4;  // independent 16-byte loads in flight per lane in the K and V passes
+// Independent 16-byte loads in flight per lane in the K and V passes; with 7
+// CTAs per SM (72 registers) six was measured faster than four at 8 CTAs and
+// than eight at 6 CTAs (OPT-30B and OPT-175B decode shapes, KV length 528
+// and 1040).
+constexpr int kUnroll = 6;
+constexpr int kMinBlocks = 7;
 
 __device__ __forceinline__ void block_reduce_stats(float (&v)[kStatN], float (*red)[kStatN]) {
 #pragma unroll
@@ -97,7 +103,7 @@ __device__ __forceinline__ void block_reduce_stats(float (&v)[kStatN], float (*r
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 8) attn_decode_q4_kernel(const __half* __restrict__ q, int ldq, KvView kv,
+__global__ void __launch_bounds__(kThreads, kMinBlocks) attn_decode_q4_kernel(const __half* __restrict__ q, int ldq, KvView kv,
                                                                   int heads, int len, __half* __restrict__ out,
                                                                   int ldo, float inv_sqrt_d, AppendRow app) {
   pdl_wait();  // q, the cache and the outputs follow the stream's earlier kernels

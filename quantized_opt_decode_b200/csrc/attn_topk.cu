@@ -8,12 +8,13 @@
 // The kept weights are the full-softmax weights, not renormalised over T;
 // with kk = L the result is dense attention.
 //
-// One CTA of 256 threads per (head, sequence).  Scores as in the dense
+// One CTA of 128 threads per (head, sequence).  Scores as in the dense
 // kernel (q as 15-bit fixed point, dp4a over the nibbles, scale*dot +
-// min*sum q per group), kept in shared memory.  The kk-th largest score is
-// found by a 4-pass radix select on an order-preserving 32-bit key (8 bits
-// per pass, a 256-bin histogram in shared memory); keys equal to it are kept
-// in index order up to kk by a block-wide prefix count.  V is token-
+// min*sum q per group), kept in shared memory.  Selection: 1024 equal-width
+// value bins over [min, max] of the scores (a monotone map, so the kk-th
+// largest score falls in the bin where the count from the top reaches kk);
+// every key above that bin is kept, and the keys inside it are ranked exactly
+// (order-preserving 32-bit key, the lower index first among equal keys).  V is token-
 // interleaved in blocks of 8 tokens, so a block is read only when it holds a
 // kept token; its weights are 16-bit fixed point normalised by the largest
 // kept p * scale of each group, 0 for the tokens not kept.
@@ -26,7 +27,8 @@
 namespace flexq {
 namespace {
 
-constexpr int kTkThreads = 256;
+constexpr int kTkThreads = 128;
+constexpr int kBins = 1024;  // kBins / kTkThreads bins per thread in the bucket search
 constexpr int kTkWarps = kTkThreads / 32;
 
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -42,6 +44,17 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   float r = 0.f;
 #pragma unroll
   for (int w = 0; w < kTkWarps; ++w) r += red[w];
+  return r;
+}
+
+__device__ __forceinline__ float block_min(float v, float* red) {
+  v = -warp_max(-v);
+  __syncthreads();
+  if (lane_id() == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kTkWarps; ++w) r = fminf(r, red[w]);
   return r;
 }
 
@@ -92,8 +105,10 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
   constexpr int DPV = D / 32;
   extern __shared__ float sc[];                                  // [len] scores
   int* blist = reinterpret_cast<int*>(sc + ((len + 3) & ~3));     // [nblk] blocks holding a kept key
-  uint8_t* sel = reinterpret_cast<uint8_t*>(blist + (((len + 7) / 8 + 3) & ~3));  // [len] kept flags
-  __shared__ int hist[256];
+  int* cand = blist + (((len + 7) / 8 + 3) & ~3);                   // [len] keys in the threshold bin
+  uint8_t* sel = reinterpret_cast<uint8_t*>(cand + ((len + 3) & ~3));  // [len] kept flags
+  __shared__ int hist[kBins];
+  __shared__ int ncand;
   __shared__ int scan[kTkWarps];
   __shared__ float red[kTkWarps];
   __shared__ float stat[2 * G + 1];
@@ -152,7 +167,7 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
   }
   // kUnroll groups of tokens are loaded before any is used, so each lane keeps
   // several loads in flight (the pass is bound by load latency otherwise)
-  float mx = -INFINITY;
+  float mx = -INFINITY, mn = INFINITY;
   constexpr int kStride = kTkThreads / 4;  // tokens per block-wide step
   constexpr int kUnroll = 4;
   for (int base = warp * 8; base < len; base += kUnroll * kStride) {
@@ -199,80 +214,80 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
         const float s = partial * inv_sqrt_d;
         if (cq == 0) sc[t] = s;
         mx = fmaxf(mx, s);
+        mn = fminf(mn, s);
       }
     }
   }
   const float M = block_max(mx, red);  // its barriers also publish sc[]
 
-  // ---- radix select: the kk-th largest key
-  uint32_t prefix = 0u, mask = 0u;
-  int need = kk;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += kTkThreads) hist[b] = 0;
-    __syncthreads();
-    // lanes that hit the same bin add once, by their lowest lane (the
-    // scores cluster in a few bins per pass, so plain atomics would serialise)
-    for (int t0 = 0; t0 < len; t0 += kTkThreads) {
-      const int t = t0 + threadIdx.x;
-      uint32_t key = 0u;
-      if (t < len) key = order_key(sc[t]);
-      const bool act = t < len && (key & mask) == prefix;
-      const int bin = act ? static_cast<int>((key >> shift) & 255u) : 256 + lane;
-      const unsigned same = __match_any_sync(0xffffffffu, bin);
-      if (act && __ffs(same) - 1 == lane) atomicAdd(&hist[bin], __popc(same));
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // the bucket b from the top with (keys above b) < need <= (keys above
-      // b) + hist[b]: lane l owns bins 8l .. 8l+7, a suffix sum over lanes
-      // finds the lane, which then walks its own bins downwards
-      int cnt[8], own = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        cnt[k] = hist[lane * 8 + k];
-        own += cnt[k];
-      }
-      int incl = own;  // keys in bins of lanes lane .. 31
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_down_sync(0xffffffffu, incl, o);
-        if (lane + o < 32) incl += n;
-      }
-      const int above_lane = incl - own;
-      const unsigned hit = __ballot_sync(0xffffffffu, above_lane < need && need <= incl);
-      if (lane == 31 - __clz(hit)) {  // the highest lane that holds the bucket
-        int above = above_lane, b = lane * 8 + 7;
-        for (int k = 7; k > 0; --k, --b) {
-          if (above + cnt[k] >= need) break;
-          above += cnt[k];
-        }
-        pick[0] = static_cast<uint32_t>(b);
-        pick[1] = static_cast<uint32_t>(above);
-      }
-    }
-    __syncthreads();
-    need -= static_cast<int>(pick[1]);
-    prefix |= pick[0] << shift;
-    mask |= 255u << shift;
-    __syncthreads();
-  }
-  const uint32_t tau = prefix;  // keys > tau are kept, and `need` of the keys == tau, lowest index first
+  const float m0 = block_min(mn, red);
 
-  // ---- kept flags; equal keys ranked in index order over contiguous segments
+  // ---- selection.  bin(t) = min(kBins-1, floor((s_t - m0) * kBins / (M - m0)))
+  // is non-decreasing in s_t (every step rounds monotonically), so the kk-th
+  // largest score lies in bin B with (keys in bins > B) < kk <= (keys in
+  // bins >= B); all scores equal puts every key in bin 0.
+  const float bscale = M > m0 ? static_cast<float>(kBins) / (M - m0) : 0.f;
+  auto bin_of = [&](float v) { return min(kBins - 1, static_cast<int>((v - m0) * bscale)); };
+  for (int b = threadIdx.x; b < kBins; b += kTkThreads) hist[b] = 0;
+  if (threadIdx.x == 0) ncand = 0;
+  __syncthreads();
+  for (int t0 = 0; t0 < len; t0 += kTkThreads) {
+    const int t = t0 + threadIdx.x;
+    const bool act = t < len;
+    const int bin = act ? bin_of(sc[t]) : kBins + lane;
+    // lanes that hit the same bin add once, by their lowest lane
+    const unsigned same = __match_any_sync(0xffffffffu, bin);
+    if (act && __ffs(same) - 1 == lane) atomicAdd(&hist[bin], __popc(same));
+  }
+  __syncthreads();
+  {
+    // thread i owns bins [kPer * i, kPer * i + kPer); a suffix sum over the
+    // threads (the block scan on reversed thread order) finds the owner of B
+    constexpr int kPer = kBins / kTkThreads;
+    const int owner = kTkThreads - 1 - threadIdx.x;  // scan order: the top bins first
+    int cnt[kPer], own = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      cnt[k] = hist[owner * kPer + k];
+      own += cnt[k];
+    }
+    int total = 0;
+    const int above = block_exclusive_scan(own, scan, &total);  // keys in the bins above this thread's
+    if (above < kk && kk <= above + own) {
+      int a = above, b = owner * kPer + kPer - 1;
+      for (int k = kPer - 1; k > 0; --k, --b) {
+        if (a + cnt[k] >= kk) break;
+        a += cnt[k];
+      }
+      pick[0] = static_cast<uint32_t>(b);
+      pick[1] = static_cast<uint32_t>(a);
+    }
+  }
+  __syncthreads();
+  const int B = static_cast<int>(pick[0]);
+  const int need = kk - static_cast<int>(pick[1]);  // keys of bin B to keep
+  for (int t = threadIdx.x; t < len; t += kTkThreads) {
+    const int bin = bin_of(sc[t]);
+    sel[t] = bin > B;
+    if (bin == B) cand[atomicAdd(&ncand, 1)] = t;
+  }
+  __syncthreads();
+  // exact rank inside bin B: keys above this one, then equal keys at a lower slot
+  const int nc = ncand;
+  for (int ci = threadIdx.x; ci < nc; ci += kTkThreads) {
+    const int t = cand[ci];
+    const uint32_t key = order_key(sc[t]);
+    int r = 0;
+    for (int cj = 0; cj < nc; ++cj) {
+      const int u = cand[cj];
+      const uint32_t ku = order_key(sc[u]);
+      r += ku > key || (ku == key && u < t);
+    }
+    sel[t] = r < need;
+  }
+  // contiguous segments for the ordered index output
   const int seg = (len + kTkThreads - 1) / kTkThreads;
   const int t0 = threadIdx.x * seg, t1 = min(len, t0 + seg);
-  int n_eq = 0;
-  for (int t = t0; t < t1; ++t) n_eq += order_key(sc[t]) == tau;
-  int total = 0;
-  int rank = block_exclusive_scan(n_eq, scan, &total);
-  int n_sel = 0;
-  for (int t = t0; t < t1; ++t) {
-    const uint32_t key = order_key(sc[t]);
-    bool keep = key > tau;
-    if (key == tau) keep = rank++ < need;
-    sel[t] = keep;
-    n_sel += keep;
-  }
 
   // ---- softmax sum over all keys; per group sum p*min and max p*scale over the kept keys
   float s_all = 0.f;
@@ -306,6 +321,8 @@ __global__ void __launch_bounds__(kTkThreads) attn_topk_q4_kernel(const __half* 
 
   // ---- kept indices in ascending order
   if (idx_out != nullptr) {
+    int n_sel = 0;
+    for (int t = t0; t < t1; ++t) n_sel += sel[t];
     int all = 0;
     int at = block_exclusive_scan(n_sel, scan, &all);
     int32_t* dst = idx_out + hr * kk;
@@ -402,7 +419,8 @@ template <int D>
 cudaError_t launch_topk(const __half* q, int ldq, const KvView& kv, int b, int heads, int len, int kk, __half* out,
                         int ldo, int32_t* idx, const AppendRow& app, cudaStream_t s) {
   const size_t smem = static_cast<size_t>((len + 3) & ~3) * sizeof(float) +
-                      static_cast<size_t>(((len + 7) / 8 + 3) & ~3) * sizeof(int) + static_cast<size_t>((len + 15) & ~15);
+                      static_cast<size_t>(((len + 7) / 8 + 3) & ~3) * sizeof(int) +
+                      static_cast<size_t>((len + 3) & ~3) * sizeof(int) + static_cast<size_t>((len + 15) & ~15);
   if (smem > 48 * 1024) {
     const cudaError_t e = cudaFuncSetAttribute(attn_topk_q4_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
