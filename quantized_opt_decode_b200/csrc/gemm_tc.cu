@@ -1202,7 +1202,7 @@ Plan make_plan(int m, int n, int k, int w_bits, int force_splits, int force_tok_
     P.tmem_alloc = 2 * cols;
   }
   const int a_slot = w_bits == 4 && !P.tmem_a ? P.ks * kATileBytes : 0;
-  P.a_stages = w_bits != 4 ? 0 : P.tmem_a ? std::min(4, static_cast<int>((512 - P.a_col0) / (32 * P.ks))) : 2;
+  P.a_stages = w_bits != 4 ? 0 : P.tmem_a ? std::min(4, static_cast<int>((512 - P.a_col0) / (32 * P.ks))) : 3;
   P.w_slot_bytes = static_cast<uint32_t>(w_bits == 4 ? round_up(P.ks * kTileBytes, 1024) : P.ks * kATileBytes);
   P.b_slot_bytes = static_cast<uint32_t>(P.ks * P.tok_tile * 128);
   const int rest = budget - P.a_stages * a_slot;

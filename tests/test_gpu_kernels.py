@@ -145,8 +145,11 @@ def test_kv_append_bit_exact(h, heads, pos0, ntok):
 
 @pytest.mark.parametrize("h,heads,kv_bits,length", [(256, 4, 4, 1), (256, 4, 4, 37), (512, 4, 4, 545),
                                                     (256, 4, 16, 33), (512, 4, 16, 300),
-                                                    (1024, 8, 4, 1030)])
+                                                    (1024, 8, 4, 1030), (256, 2, 4, 12000)])
 def test_attention_decode(h, heads, kv_bits, length):
+    """Dense decode attention against the oracle; d = 64 and 128, ragged
+    8-token blocks, and (12000 slots at d = 128) a cache too long for its V
+    (min, scale) pairs to be gathered into shared memory."""
     cfg = _cfg(h, heads, kv_bits)
     b, L = 3, length + 3
     rng = np.random.default_rng(length + h)
