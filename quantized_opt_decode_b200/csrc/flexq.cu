@@ -264,10 +264,9 @@ bool decode_fusable(int b) { return b >= 1 && b <= kFuseMaxRows; }
 
 // Decode step of one layer for b sequences, fused ([WT] "P/D阶段计算",
 // decoding phase): u_in = LN1(t) computed by the caller (the previous
-// layer's FC2 or the embedding); the QKV projection's epilogue puts this
-// token's K/V straight into cache slot pos (fp16 rows, or quantized on
-// append into the 4-bit cache) and the decode attention reads slots
-// 0..pos; the output
+// layer's FC2 or the embedding); the QKV projection stores this token's K/V
+// straight into an fp16 cache slot pos, or the decode attention quantizes
+// them into a 4-bit cache slot pos before it reads slots 0..pos; the output
 // projection adds the residual and LayerNorms its rows (LN2) after a grid
 // barrier; FC1 + GELU; FC2 adds the residual and, when ln_next_g is set,
 // LayerNorms its rows into u_out (the next layer's LN1 or the final LN).
@@ -278,29 +277,27 @@ flexq_status decode_fused(const flexq_config* c, const flexq_layer* L, const __h
   const int h = c->h, f = c->ffn, d = h / c->heads;
   const KvView kvv = view_of(c, kv, seq0);
   int* tile_ctr = w.tile_ctr;
-  // the QKV epilogue writes the token's K/V into cache slot pos (4-bit:
-  // quantized on append), so the attention reads the cache as it stands
   KvFuse kf{};
-  kf.bits = c->kv_bits;
+  AppendRow app = kNoAppend;
   if (c->kv_bits == 16) {
     kf.k = static_cast<__half*>(kvv.k);
     kf.v = static_cast<__half*>(kvv.v);
+    kf.h = h;
+    kf.heads = c->heads;
+    kf.d = d;
+    kf.max_len = kvv.max_len;
+    kf.pos = pos;
   } else {
-    kf.kq = static_cast<uint8_t*>(kvv.k);
-    kf.vq = static_cast<uint32_t*>(kvv.v);
-    kf.kmeta = static_cast<__half2*>(kvv.k_meta);
-    kf.vmeta = static_cast<__half2*>(kvv.v_meta);
+    app.k = w.qkv + h;
+    app.v = w.qkv + 2 * h;
+    app.ld = 3 * h;
+    app.pos = pos;
   }
-  kf.h = h;
-  kf.heads = c->heads;
-  kf.d = d;
-  kf.max_len = kvv.max_len;
-  kf.pos = pos;
-  const AppendRow app = kNoAppend;
   {
     ProfScope ps(FLEXQ_K_QKV, s);
     FQ_TRY(run_linear(u_in, h, L->w_qkv, c->w_bits, b, 3 * h, h, static_cast<const __half*>(L->b_qkv), nullptr, 0,
-                      EPI_BIAS, w.qkv, 3 * h, w.acc, w.acc_bytes, s, "QKV projection", &kf, nullptr, tile_ctr));
+                      EPI_BIAS, w.qkv, 3 * h, w.acc, w.acc_bytes, s, "QKV projection",
+                      c->kv_bits == 16 ? &kf : nullptr, nullptr, tile_ctr));
   }
   {
     ProfScope ps(FLEXQ_K_ATTN_DECODE, s);

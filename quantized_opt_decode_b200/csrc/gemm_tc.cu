@@ -65,9 +65,7 @@ constexpr int kATileBytes = 128 * 64 * 2;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr int kBarrierBytes = 1024;  // mbarriers, TMEM address, flags, finalize slot list
 constexpr int kMaxBarriers = 56;     // mbarriers fit in the first 448 bytes of that region
-// per epilogue warp: 16 tokens x 33 floats of transpose stage, then the 4-bit
-// KV append's group (min, max) exchange: 2 chunks x 4 warps x 16 tokens x 2
-constexpr int kEpiStageBytes = 4 * 16 * 33 * 4 + 2 * 4 * 16 * 2 * 4;
+constexpr int kEpiStageBytes = 4 * 16 * 33 * 4;  // per epilogue warp: 16 tokens x 33 floats
 constexpr int kMaxWStages = 16;
 constexpr int kMinItersPerCta = 8;
 constexpr int kMaxContrib = 64;
@@ -111,7 +109,7 @@ struct GemmParams {
   int* counters;    // [tiles][2]: contributors arrived, partials published
   uint64_t wait_ns;
   uint32_t* err;
-  int kv_on;        // decode QKV: K/V tiles go to the cache (fp16 rows, or quantized on append)
+  int kv_on;        // decode QKV: K/V tiles go to the fp16 cache
   KvFuse kv;
   int ln_on;        // decode out-proj / FC2: LayerNorm of the rows after a grid barrier
   LnFuse ln;
@@ -330,7 +328,6 @@ struct Ctl {
   volatile int* fin_me;
   int* fin_slots;  // [kMaxContrib]
   float* stage;    // [4][16][33]
-  float* grp;      // [2][4][16][2]
 };
 
 __device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
@@ -344,7 +341,6 @@ __device__ __forceinline__ Ctl make_ctl(uint8_t* region, uint64_t* accf) {
   c.fin_me = c.abort_flag + 3;
   c.fin_slots = reinterpret_cast<int*>(region + kBarrierBytes / 2);
   c.stage = reinterpret_cast<float*>(region + kBarrierBytes);
-  c.grp = c.stage + 4 * 16 * 33;
   return c;
 }
 
@@ -382,91 +378,6 @@ __device__ __forceinline__ void acc_load16(const GemmParams& p, uint32_t tbase, 
   }
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* ptr) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
-// The 4-bit cache's V word of (sequence tok, head, dimension e) in the 8-token
-// block that holds slot pos.
-__device__ __forceinline__ uint32_t* kv_vword(const KvFuse& kv, int tok, int head, int e) {
-  return kv.vq + ((static_cast<size_t>(tok) * kv.heads + head) * (kv_pad_len(kv.max_len) / 8) + kv.pos / 8) * kv.d + e;
-}
-
-// Quantize on append inside the QKV epilogue (4-bit cache): this lane holds
-// 16 consecutive features (head dimensions e0..e0+15) of token tok, x = the
-// fp32 accumulators before bias in the transpose stage; the fp16 K/V value is
-// the rounding of x + bias, as the projection's output would hold it.  A
-// 64-element group is spread over two warps (qd and qd ^ 1) x two lanes
-// (hf 0, 1): min and max by one shuffle and one exchange through shared
-// memory (a barrier of the four epilogue warps, so every epilogue thread
-// calls this), then the codec's rounding (fp32 scale = (max - min) / 15
-// rounded to fp16, min to fp16, codes rint((v - min) / scale) clamped to
-// 0..15).  K: 8 bytes of canonical codes; V: the token's nibble merged into
-// its 16 token-interleaved words (vold, read earlier from vdst); the group's
-// first lane writes its (min, scale).  The values are re-read from the stage
-// rather than held, to keep the epilogue's registers down.
-__device__ __forceinline__ float kv_value(const float* x, const float (&bv)[16], int u) {
-  return __half2float(__float2half_rn(x[u] + bv[u]));
-}
-
-__device__ __forceinline__ uint32_t kv_code(float v, float mn, float sc) {
-  if (sc == 0.0f) return 0u;
-  return static_cast<uint32_t>(fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(v, mn), sc)), 0.0f), 15.0f));
-}
-
-__device__ __forceinline__ void kv_append_q4(const GemmParams& p, const Ctl& c, const float* x, const float (&bv)[16],
-                                             int tok, int par, int qd, int jt, int hf, bool is_v, int head, int e0,
-                                             uint4 (&vold)[4], uint4* vdst) {
-  float lo = INFINITY, hi = -INFINITY;
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const float v = kv_value(x, bv, u);
-    lo = fminf(lo, v);
-    hi = fmaxf(hi, v);
-  }
-  lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, 1));
-  hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, 1));
-  float* gx = c.grp + par * (4 * 16 * 2);
-  if (hf == 0) {
-    gx[(qd * 16 + jt) * 2] = lo;
-    gx[(qd * 16 + jt) * 2 + 1] = hi;
-  }
-  epi_bar();
-  lo = fminf(lo, gx[((qd ^ 1) * 16 + jt) * 2]);
-  hi = fmaxf(hi, gx[((qd ^ 1) * 16 + jt) * 2 + 1]);
-  if (tok >= p.m) return;
-  lo = __fadd_rn(lo, 0.0f);  // -0 -> +0
-  hi = __fadd_rn(hi, 0.0f);
-  const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
-  const __half m16 = __float2half_rn(lo);
-  const float sc = __half2float(s16);
-  const float mn = __half2float(m16);
-  const KvFuse& kv = p.kv;
-  const size_t slot = (static_cast<size_t>(tok) * kv.heads + head) * kv.max_len + kv.pos;
-  if (!is_v) {
-    uint32_t w0 = 0u, w1 = 0u;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      w0 |= kv_code(kv_value(x, bv, e), mn, sc) << (4 * e);
-      w1 |= kv_code(kv_value(x, bv, 8 + e), mn, sc) << (4 * e);
-    }
-    *reinterpret_cast<uint2*>(kv.kq + slot * (kv.d / 2) + e0 / 2) = make_uint2(w0, w1);
-  } else {
-    const int sh = 4 * (kv.pos & 7);
-    const uint32_t keep = ~(0xFu << sh);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      vold[u].x = (vold[u].x & keep) | (kv_code(kv_value(x, bv, 4 * u), mn, sc) << sh);
-      vold[u].y = (vold[u].y & keep) | (kv_code(kv_value(x, bv, 4 * u + 1), mn, sc) << sh);
-      vold[u].z = (vold[u].z & keep) | (kv_code(kv_value(x, bv, 4 * u + 2), mn, sc) << sh);
-      vold[u].w = (vold[u].w & keep) | (kv_code(kv_value(x, bv, 4 * u + 3), mn, sc) << sh);
-      vdst[u] = vold[u];
-    }
-  }
-  if ((qd & 1) == 0 && hf == 0)
-    (is_v ? kv.vmeta : kv.kmeta)[slot * (kv.d / 64) + e0 / 64] = __halves2half2(m16, s16);
-}
-
 __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_base, int warp, int lane) {
   pdl_wait();  // the residual, outputs, partials and counters belong to the stream's order
   const Sched& sc = p.sc;
@@ -481,24 +392,6 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
     int buf;
     uint32_t par;
     acc_slot(q, p.acc_bufs, buf, par);
-    const int n_tile = g.tile % sc.n_tiles;
-    const int tok0 = (g.tile / sc.n_tiles) * p.tok_tile;
-    const int f_out = n_tile * 128 + qd * 32 + hf * 16;  // features this lane finishes
-    // decode QKV: the K and V tiles go to the cache slot instead of the output
-    const bool kv_tile = p.kv_on && n_tile * 128 >= p.kv.h;
-    const bool kv_v = kv_tile && f_out >= 2 * p.kv.h;
-    const int kv_cc = kv_tile ? f_out - (kv_v ? 2 * p.kv.h : p.kv.h) : 0;
-    const int kv_head = kv_tile ? kv_cc / p.kv.d : 0;
-    const int kv_e0 = kv_tile ? kv_cc % p.kv.d : 0;  // first of this lane's 16 head dimensions
-    const bool kv_q4 = kv_tile && p.kv.bits == 4;
-    // 4-bit V: the token's nibble is merged into words that hold 7 earlier
-    // tokens; bring those lines into L2 while the tile's MMAs run
-    if (kv_q4 && kv_v && hf == 0) {
-      for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
-        const int tok = tok0 + c0 + jt;
-        if (tok < p.m) prefetch_l2(kv_vword(p.kv, tok, kv_head, kv_e0));
-      }
-    }
     const bool ok = mbar_wait(&c.accf[buf], par, drain_ns(p.wait_ns));
     if (!ok) set_error(p.err, DEV_TIMEOUT_EPILOGUE);
     tc_fence_after();
@@ -508,8 +401,13 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       mbar_arrive(&c.acce[buf]);
       continue;
     }
+    const int n_tile = g.tile % sc.n_tiles;
+    const int tok0 = (g.tile / sc.n_tiles) * p.tok_tile;
     const uint32_t tbase =
         tmem_base + static_cast<uint32_t>(buf) * p.acc_cols + (static_cast<uint32_t>(qd * 32) << 16);
+    const int f_out = n_tile * 128 + qd * 32 + hf * 16;  // features this lane finishes
+    // decode QKV with an fp16 cache: the K and V tiles go to the cache slot
+    const bool kv_tile = p.kv_on && n_tile * 128 >= p.kv.h;
     // Split tile: count in; the last to arrive finishes the tile.
     int ns = 1, me = 0;
     if (!g.full) {
@@ -572,15 +470,6 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       for (int j = 0; j < 16; ++j) nxt[j] = __ldcg(other + j * 128 + frow);
     }
     for (int c0 = 0; c0 < p.tok_tile; c0 += 16) {
-      // 4-bit V: this lane's 16 words of the token's 8-token block, loaded
-      // before the accumulator so the read overlaps it
-      uint4 vold[4];
-      uint4* vdst = nullptr;
-      if (kv_q4 && kv_v && tok0 + c0 + jt < p.m) {
-        vdst = reinterpret_cast<uint4*>(kv_vword(p.kv, tok0 + c0 + jt, kv_head, kv_e0));
-#pragma unroll
-        for (int u = 0; u < 4; ++u) vold[u] = __ldcg(vdst + u);
-      }
       float acc[16];
       float v[16];
       if (one_other) {
@@ -620,10 +509,7 @@ __device__ void epilogue_role(const GemmParams& p, const Ctl& c, uint32_t tmem_b
       for (int j = 0; j < 16; ++j) stg[j * 33 + lane] = v[j];
       __syncwarp();
       const int tok = tok0 + c0 + jt;
-      if (kv_q4) {
-        kv_append_q4(p, c, stg + jt * 33 + hf * 16, bv, tok, (c0 >> 4) & 1, qd, jt, hf, kv_v, kv_head, kv_e0,
-                     vold, vdst);
-      } else if (kv_tile) {
+      if (kv_tile) {
         // this lane's 16 features of its token (+ bias) go to slot pos
         if (tok < p.m) {
           uint32_t packed[8];
@@ -1445,7 +1331,7 @@ cudaError_t launch_linear(const LinearArgs& a, void* ws, size_t ws_bytes, cudaSt
   if (a.kv != nullptr) {
     // whole 64-feature groups of one head per K/V tile; one token tile
     if (a.m > kFuseMaxRows || P.tok_tiles != 1 || a.n != 3 * a.kv->h || a.kv->h % 128 != 0 ||
-        (a.epi & ~EPI_BIAS) != 0 || a.kv->d % 64 != 0 || (a.kv->bits != 16 && a.kv->bits != 4))
+        (a.epi & ~EPI_BIAS) != 0)
       return cudaErrorInvalidValue;
     p.kv_on = 1;
     p.kv = *a.kv;

@@ -102,21 +102,15 @@ enum Epilogue : int {
   EPI_F32_OUT = 8,    // write fp32 (no bias/act/residual allowed)
 };
 // Decode-step fusions of a linear layer (one token per sequence, m rows):
-// KvFuse makes the QKV projection put its K and V columns straight into
-// cache slot `pos` of each of the m sequences instead of its output: the
-// fp16 rows, or (bits 4) the rows quantized on append, codes and (min, scale)
-// exactly as the codec makes them of the fp16 rows;
+// KvFuse makes the QKV projection store its K and V columns straight into
+// the fp16 cache slot `pos` of each of the m sequences instead of its output
+// (a 4-bit cache is appended by the decode attention, see AppendRow);
 // LnFuse makes the layer LayerNorm its finished rows [m][n] into `y` after a
 // grid-wide barrier (the launch is cooperative; `sync` = two ints of device
 // memory that are zero on entry and left zero).
 struct KvFuse {
-  int bits;         // 16 or 4
-  __half* k;        // 16: fp16 caches in the KvView layout of the m sequences
+  __half* k;  // fp16 caches in the KvView layout of the m sequences
   __half* v;
-  uint8_t* kq;      // 4: K codes [m][heads][max_len][d/2]
-  uint32_t* vq;     // 4: V words [m][heads][kv_pad_len(max_len)/8][d]
-  __half2* kmeta;   // 4: (min, scale) [m][heads][max_len][d/64]
-  __half2* vmeta;
   int h, heads, d, max_len, pos;
 };
 struct LnFuse {
