@@ -74,9 +74,10 @@ def csrc_hash(files=None):
 # Source files that define each kernel kind's device code: an ncu traffic
 # figure stays valid while these are unchanged.
 _SHARED = ["common.cuh", "kernels.h"]
-_GEMM = ["gemm_tc.cu", "quant_common.cuh"] + _SHARED  # the decode QKV epilogue quantizes K/V
+_GEMM = ["gemm_tc.cu"] + _SHARED
 KERNEL_FILES = {
-    "attn_decode": ["attn_decode.cu", "attn_topk.cu"] + _SHARED,
+    # the decode attention kernels quantize the appended token with quant_common.cuh
+    "attn_decode": ["attn_decode.cu", "attn_topk.cu", "quant_common.cuh"] + _SHARED,
     "qkv": _GEMM, "out_proj": _GEMM, "fc1": _GEMM, "fc2": _GEMM, "lm_head": _GEMM,
     "kv_append": ["kv_append.cu", "quant_common.cuh"] + _SHARED,
     "layernorm": ["rowwise.cu"] + _SHARED, "embed": ["rowwise.cu"] + _SHARED,

@@ -32,6 +32,22 @@ __device__ __forceinline__ void load32(const __half* p, float (&v)[32], bool val
   }
 }
 
+// code = clamp(rint(a / s), 0, 15) with a / s the correctly rounded fp32
+// quotient, computed without a division in almost every case: r = a * fl(1/s)
+// differs from fl(a / s) by less than |r| * 2^-22 (two roundings of relative
+// size 2^-24 in r, one in the quotient), so wherever r is farther than
+// |r| * 2^-20 (plus 2^-40) from a rounding boundary k + 1/2, both round to
+// the same integer k; only a value that close takes the exact quotient.  r - k
+// and 1/2 - |r - k| are exact in fp32 (Sterbenz), so the test itself does not
+// round.  s > 0.
+__device__ __forceinline__ uint32_t q64_code(float a, float s, float inv_s) {
+  const float r = __fmul_rn(a, inv_s);
+  float k = rintf(r);
+  const float margin = __fadd_rn(__fmul_rn(fabsf(r), 0x1p-20f), 0x1p-40f);
+  if (fabsf(__fsub_rn(0.5f, fabsf(__fsub_rn(r, k)))) <= margin) k = rintf(__fdiv_rn(a, s));
+  return static_cast<uint32_t>(fminf(fmaxf(k, 0.0f), 15.0f));
+}
+
 // Quantizes one 64-element group held by a lane pair (lanes 2i and 2i+1 of the
 // warp, 32 elements each).  Every lane of the warp must call this.
 __device__ __forceinline__ void q64_lane_pair(const float (&v)[32], uint32_t (&q)[32], __half& m16,
@@ -50,12 +66,9 @@ __device__ __forceinline__ void q64_lane_pair(const float (&v)[32], uint32_t (&q
   m16 = __float2half_rn(lo);
   const float s = __half2float(s16);
   const float m = __half2float(m16);
+  const float inv_s = s != 0.0f ? __frcp_rn(s) : 0.0f;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    float r = 0.0f;
-    if (s != 0.0f) r = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(v[e], m), s)), 0.0f), 15.0f);
-    q[e] = static_cast<uint32_t>(r);
-  }
+  for (int e = 0; e < 32; ++e) q[e] = s != 0.0f ? q64_code(__fsub_rn(v[e], m), s, inv_s) : 0u;
 }
 
 // 8 codes -> one 32-bit word, nibble e holds element e (low nibble = even

@@ -46,6 +46,45 @@ def test_quantize_bit_exact(n_groups):
     assert np.array_equal(to_host(out).view(np.uint16), q64.dequantize(c_ref, m_ref, s_ref).view(np.uint16))
 
 
+def _boundary_groups(rng, n_groups):
+    """Groups whose quotients (x - min) / scale sit on or one fp16 step beside
+    the half-integers where rint changes its result: exact ties (half to even)
+    and values a reciprocal multiply alone would round the other way."""
+    x = np.empty((n_groups, 64), dtype=np.float16)
+    for g in range(n_groups):
+        s = np.float16(rng.choice([3, 5, 7, 11, 13, 0.75, 1 / 3, 0.1, 0.7]) if g % 2 == 0
+                       else np.exp(rng.uniform(-7, 2)))
+        m = np.float16(rng.choice([0.0, -1.5, 2.25, -7.0]) if g % 3 else rng.standard_normal())
+        vals = [m, np.float16(np.float32(m) + 15 * np.float32(s))]
+        while len(vals) < 64:
+            v = np.float16(np.float32(m) + (rng.integers(0, 15) + 0.5) * np.float32(s))
+            vals += [v, np.nextafter(v, np.float16(np.inf)), np.nextafter(v, np.float16(-np.inf))]
+        x[g] = np.array(vals[:64], dtype=np.float16)
+    return x.reshape(-1)
+
+
+@pytest.mark.parametrize("kind", ["boundaries", "subnormal"])
+def test_quantize_rounding_boundaries_bit_exact(kind):
+    """Codes at and next to the rounding boundaries of rint((x - min) / scale),
+    where the quotient must be the correctly rounded fp32 one (in the boundary
+    set, rounding a * (1/scale) instead changes about 0.5 % of the codes), and
+    groups of fp16 subnormals (coarse grids, many exact ties)."""
+    rng = np.random.default_rng(11 if kind == "boundaries" else 12)
+    if kind == "boundaries":
+        x = _boundary_groups(rng, 2048)
+    else:
+        x = (rng.standard_normal(64 * 4096) * 1e-6).astype(np.float16)
+    n = x.size
+    codes = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    mn = torch.empty(n // 64, dtype=torch.float16, device="cuda")
+    sc = torch.empty(n // 64, dtype=torch.float16, device="cuda")
+    fq.flexq_quantize(to_dev(x), n, codes, mn, sc)
+    c_ref, m_ref, s_ref = q64.quantize(x)
+    assert np.array_equal(to_host(codes), c_ref)
+    assert np.array_equal(to_host(mn).view(np.uint16), m_ref.view(np.uint16))
+    assert np.array_equal(to_host(sc).view(np.uint16), s_ref.view(np.uint16))
+
+
 def test_dequantize_every_code_and_byte():
     """All 256 byte values under random (min, scale) pairs."""
     rng = np.random.default_rng(9)
