@@ -299,10 +299,12 @@ flexq_status flexq_layer_prefill(const flexq_config* cfg, const flexq_layer* lay
  * y_dev fp16 [b][h] (distinct).  Appends this token's K/V to slot pos, then
  * attends over slots 0..pos read back from the cache.  For b <= 256 the
  * append needs no launch of its own: a 4-bit cache is appended by the
- * decode attention kernel (one warp of each (sequence, head) CTA quantizes
- * the token's K/V rows, the same codes flexq_kv_append gives those fp16
- * rows, before the CTA reads the cache), an fp16 cache by the Q/K/V
- * projection's epilogue; LN2 runs inside the output projection (a
+ * decode attention kernel (the warps of each (sequence, head) CTA quantize
+ * the token's K/V rows, one warp per 64-element group, the same codes
+ * flexq_kv_append gives those fp16 rows, before the CTA reads the cache;
+ * when the attention splits each head's cache over several CTAs the append
+ * is a launch of its own), an fp16 cache by the Q/K/V projection's
+ * epilogue; LN2 runs inside the output projection (a
  * cooperative launch whose CTAs normalise the finished rows after a
  * grid-wide barrier); decode attention splits each head's cache over several
  * CTAs when b * heads CTAs would not fill the GPU. */
