@@ -165,3 +165,41 @@ def test_prefill_cache_rejects_bad_arguments(fq):
     st = fq._lib.flexq_attention_prefill_cache(C.byref(cfg), C.byref(kv), 0x1000, 256, 4, 16, 4, 0x2000, 256,
                                                None)
     assert st == 1 and "pos0" in fq.flexq_last_error()
+
+
+def test_linear_rejects_bad_arguments(fq):
+    lib = fq._lib
+    A = 0x100000  # 16-byte aligned placeholders; nothing is launched on a rejection
+    st = lib.flexq_linear(A, 64, A, 8, 4, 128, 64, None, None, 0, 0, A, 128, None, 0, 0, None)
+    assert st == 1 and "w_bits" in fq.flexq_last_error()
+    st = lib.flexq_linear(A, 96, A, 4, 4, 128, 96, None, None, 0, 0, A, 128, None, 0, 0, None)
+    assert st == 1 and "multiple of 64" in fq.flexq_last_error()
+    st = lib.flexq_linear(A + 2, 64, A, 4, 4, 128, 64, None, None, 0, 0, A, 128, None, 0, 0, None)
+    assert st == 1 and "alignment" in fq.flexq_last_error()
+    st = lib.flexq_linear(A, 64, A, 4, 4, 128, 64, None, None, 0, 1, A, 128, None, 0, 0, None)
+    assert st == 1 and "bias" in fq.flexq_last_error()
+    st = lib.flexq_linear(A, 64, A, 4, 4, 128, 64, A, None, 0, 8 | 1, A, 128, None, 0, 0, None)
+    assert st == 1 and "fp32 output" in fq.flexq_last_error()
+    st = lib.flexq_linear(A, 64, A, 4, 4, 128, 64, None, None, 0, 0, A, 128, None, 0, 2, None)
+    assert st == 1 and "force_splits" in fq.flexq_last_error()
+
+
+def test_kv_append_and_attention_reject_bad_arguments(fq):
+    cfg = fq.flexq_config(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=4, ln_eps=1e-5)
+    kv = fq.flexq_kv(0x1000, 0x2000, 0x3000, 0x4000, 4, 40)
+    lib, A = fq._lib, 0x100000
+    st = lib.flexq_kv_append(C.byref(cfg), C.byref(kv), A, A, 768, 4, 38, 3, None)
+    assert st == 1 and "outside max_len" in fq.flexq_last_error()
+    st = lib.flexq_attention_decode(C.byref(cfg), C.byref(kv), A, 768, 4, 41, A, 256, None)
+    assert st == 1 and "max_len" in fq.flexq_last_error()
+    st = lib.flexq_attention_decode(C.byref(cfg), C.byref(kv), A, 770, 4, 16, A, 256, None)
+    assert st == 1 and "strides" in fq.flexq_last_error()
+    long_kv = fq.flexq_kv(0x1000, 0x2000, 0x3000, 0x4000, 4, 20000)
+    st = lib.flexq_attention_decode(C.byref(cfg), C.byref(long_kv), A, 768, 4, 16385, A, 256, None)
+    assert st == 1 and "16384" in fq.flexq_last_error()
+    st = lib.flexq_attention_decode_topk(C.byref(cfg), C.byref(kv), A, 768, 4, 16, 17, A, 256, None, None)
+    assert st == 1 and "k must" in fq.flexq_last_error()
+    cfg16 = fq.flexq_config(h=256, heads=4, ffn=1024, w_bits=4, kv_bits=16, ln_eps=1e-5)
+    kv16 = fq.flexq_kv(0x1000, 0x2000, None, None, 4, 40)
+    st = lib.flexq_attention_decode_topk(C.byref(cfg16), C.byref(kv16), A, 768, 4, 16, 2, A, 256, None, None)
+    assert st == 1 and "4-bit" in fq.flexq_last_error()
